@@ -1,0 +1,123 @@
+// Internal launchers shared by the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "csa2.h"
+
+namespace csa2 {
+
+// Aligned carving of the caller's workspace.
+struct Carver {
+  char* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <class T>
+  T* take(size_t n) {
+    used = (used + 255) & ~size_t(255);
+    T* p = base ? reinterpret_cast<T*>(base + used) : nullptr;
+    used += n * sizeof(T);
+    return p;
+  }
+};
+
+// Radix top-k scratch for nq queries and up to two thresholds per query.
+struct TopkScratch {
+  uint32_t* hist;        // [nq][kBuckets]                 (zeroed before the histogram pass)
+  uint32_t* chunk_cnt;   // [nq][2][n_chunks]              members per chunk
+  uint64_t* cand;        // [nq][2][cand_cap]              threshold-bucket candidates
+  uint32_t* cand_cnt;    // [nq][2]
+  uint64_t* kth;         // [nq][2]                        key of the k-th best candidate
+  int32_t* thresh;       // [nq][2][2]                     bucket b*, members above b*
+  int32_t n_chunks;
+  int32_t cand_cap;
+};
+constexpr int kChunk = 4096;          // positions per chunk in the multi-CTA passes
+constexpr int kCandCap = 16384;       // threshold-bucket candidates kept per (query, k)
+
+size_t topk_scratch_bytes(int32_t nq, int32_t n_max);
+TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);
+
+// K1: scores of every visible position for every query (tcgen05 int8), plus
+// the bucket histogram.  hist may be NULL.
+cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
+                               const int32_t* seq_of_query, const int32_t* query_pos,
+                               int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
+                               int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
+                               cudaStream_t st);
+
+// Radix top-k over score rows.  ks[0..n_k) are the wanted counts (n_k <= 2,
+// ks[0] >= ks[1]); outputs go to out_idx[t]/out_cnt[t].  If hist_ready, the
+// histogram in `s.hist` is already filled (by K1); otherwise it is built here.
+struct TopkOut {
+  int32_t* idx;
+  int32_t* cnt;
+  int32_t k;
+};
+cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* n_valid,
+                              const int32_t* query_pos, const int32_t* cand_pos, int32_t nq,
+                              int32_t n_max, const TopkOut* outs, int32_t n_k,
+                              const TopkScratch& s, bool hist_ready, int32_t* status,
+                              cudaStream_t st);
+
+// Single-CTA-per-query top-k for up to kSmallMax candidates.
+constexpr int kSmallMax = 16384;
+cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* n_valid,
+                              const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
+                              int32_t* out_idx, int32_t* out_cnt, int32_t* status,
+                              cudaStream_t st);
+
+// K3 scoring part: scores of the pool entries (slot order) for each query.
+cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
+                                 const int32_t* seq_of_query, const int32_t* pool_idx,
+                                 const int32_t* pool_cnt, int32_t nq, int32_t H, int32_t D,
+                                 int32_t P, int32_t* scores, int32_t* status, cudaStream_t st);
+
+// K4: FP4 sparse attention.
+size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
+cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,
+                               const int32_t* seq_of_query, const int32_t* query_pos,
+                               const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq,
+                               int32_t Hq, int32_t D, int32_t K, int32_t window, float scale,
+                               uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                               int32_t* status, cudaStream_t st);
+
+// K7: FP4 quantiser.
+cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_x,
+                                const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes,
+                                uint8_t* scales, int64_t ld_scales, int64_t n_dst_rows,
+                                int32_t* status, cudaStream_t st);
+
+int sm_count();
+
+// Raises a kernel's dynamic shared-memory limit once per device.
+template <class F>
+cudaError_t ensure_smem(F* kernel, int bytes, unsigned long long& done_mask) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && ((done_mask >> dev) & 1ull)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && dev < 64) done_mask |= 1ull << dev;
+  return e;
+}
+
+// Attention jobs that share shapes, positions and sizes (one per layer).
+struct AttnJobDesc {
+  const uint16_t* q;
+  const csa2_rows* codes;
+  const csa2_rows* scales;
+  const int32_t* sel_idx;
+  const int32_t* sel_cnt;
+  uint16_t* out;
+  float* lse;
+};
+constexpr int kMaxAttnJobs = 16;
+cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const int32_t* seq_of_query,
+                                    const int32_t* query_pos, int32_t nq, int32_t Hq, int32_t D,
+                                    int32_t K, int32_t window, float scale, void* ws, int32_t* status,
+                                    cudaStream_t st);
+
+}  // namespace csa2

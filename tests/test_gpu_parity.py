@@ -1,0 +1,296 @@
+"""GPU parity: libcsa2 (through its C ABI) against the CPU oracle.
+
+Indices, scores and FP4 codes must match bit-exactly.  Attention outputs must
+satisfy |gpu - ref| <= 2e-3 + 1e-2 |ref| against the fp64 oracle.  These sizes
+finish in seconds on the oracle and still span several tiles and a ragged
+tail.  Full-size cases are in test_gpu_fullsize.py.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from kv_cache_decode_csa2_b200 import csa2 as B
+from tests import gpu_cases as G
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+# ------------------------------------------------------------------ K7 quantiser
+def test_fp4_quantize_bitexact():
+    rng = np.random.default_rng(0)
+    x = rng.standard_normal((2048, 512)).astype(np.float32)
+    x[::7] *= 8
+    x[1, :32] = 0                                  # zero block
+    x[2, :32] *= 1e-5                              # underflowing scale
+    x[3, :32] *= 5000                              # saturating scale
+    # exact ties of the E2M1 grid at scale 1: amax 6 pins the scale to 1.0
+    x[4, :32] = np.array([6, .25, .75, 1.25, 1.75, 2.5, 3.5, 5, -.25, -.75, -1.25, -1.75, -2.5, -3.5, -5,
+                          0, -0.0, 6, -6, 7, 1, 2, 3, 4, .5, 1.5, -1, -2, -3, -4, -.5, -1.5], np.float32)
+    # exact E4M3 ties of amax/6: midpoints between adjacent scale values
+    v = O.e4m3_decode(np.arange(0x7F))
+    mids = (v[:-1] + v[1:]) / 2 * 6
+    for i in range(32):
+        x[5 + i, :32] = 0
+        x[5 + i, 0] = mids[i * 4]
+    codes_ref, scales_ref = O.fp4_quantize(x)
+    xd = torch.from_numpy(x).to(DEV)
+    codes = torch.zeros((2048, 256), dtype=torch.uint8, device=DEV)
+    scales = torch.zeros((2048, 16), dtype=torch.uint8, device=DEV)
+    st = B.csa2_fp4_quantize(xd, codes, scales)
+    B.check_status(st)
+    assert np.array_equal(_np(scales), scales_ref)
+    assert np.array_equal(_np(codes), codes_ref)
+
+
+def test_fp4_quantize_scatter_rows():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((100, 128)).astype(np.float32)
+    dst = rng.permutation(300)[:100].astype(np.int32)
+    codes = torch.zeros((300, 64), dtype=torch.uint8, device=DEV)
+    scales = torch.zeros((300, 4), dtype=torch.uint8, device=DEV)
+    B.check_status(B.csa2_fp4_quantize(torch.from_numpy(x).to(DEV), codes, scales,
+                                       dst_rows=torch.from_numpy(dst).to(DEV)))
+    cr, sr = O.fp4_quantize(x)
+    assert np.array_equal(_np(codes)[dst], cr) and np.array_equal(_np(scales)[dst], sr)
+    untouched = np.setdiff1d(np.arange(300), dst)
+    assert not _np(codes)[untouched].any()
+
+
+# ------------------------------------------------------------------ K1 + K2: full index
+def _index_case(wl, nq_check=None):
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    nq = len(c.query_pos)
+    scores = torch.full((nq, c.max_ctx), -123, dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_index_full(ly.q, ly.w, ly.keys, c.pos_dev, c.max_ctx, seq_of_query=c.seq_dev,
+                                     scores=scores, P=wl.pool, pool_idx=ly.pool_idx, pool_cnt=ly.pool_cnt,
+                                     K=wl.topk, sel_idx=ly.sel_idx, sel_cnt=ly.sel_cnt))
+    sc, pool, pcnt, sel, scnt = map(_np, (scores, ly.pool_idx, ly.pool_cnt, ly.sel_idx, ly.sel_cnt))
+    for i in range(nq if nq_check is None else nq_check):
+        s = int(c.seq_of_query[i])
+        pos = int(c.query_pos[i])
+        q, w = c.host_q[(0, i)]
+        ref_s, ref_pool, ref_sel = O.full_index(q, w, c.host_keys[(0, s)], pos, wl.pool, wl.topk)
+        assert np.array_equal(sc[i, :pos + 1], ref_s), f"scores of query {i}"
+        assert (sc[i, pos + 1:] == -123).all()
+        assert pcnt[i] == len(ref_pool) and np.array_equal(pool[i, :pcnt[i]], ref_pool)
+        assert (pool[i, pcnt[i]:] == -1).all()
+        assert scnt[i] == len(ref_sel) and np.array_equal(sel[i, :scnt[i]], ref_sel)
+        assert (sel[i, scnt[i]:] == -1).all()
+
+
+def test_index_full_tiny_d64():
+    _index_case(synth.C0_TINY)
+
+
+def test_index_full_ragged_tail_large_path():
+    # 20011 positions: many 128-row tiles, a ragged last tile, the multi-CTA top-k
+    _index_case(synth.scaled(synth.C1_SINGLE, seq_lens=(20011,)))
+
+
+@pytest.mark.parametrize("ctx", [1, 2, 100, 129, 1025])
+def test_index_full_short_contexts(ctx):
+    # context shorter than the pool, the selection and the window
+    _index_case(synth.scaled(synth.C0_TINY, seq_lens=(ctx,)))
+
+
+def test_index_full_paged_ragged_batch():
+    wl = synth.scaled(synth.C3_RAGGED, ragged=(5, 3000, 40000))
+    _index_case(wl)
+
+
+def test_index_score_range_error():
+    q = torch.full((1, 64, 128), -128, dtype=torch.int8, device=DEV)
+    w = torch.full((1, 64), 127, dtype=torch.int8, device=DEV)
+    keys = torch.zeros((256, 128), dtype=torch.int8, device=DEV)
+    st = B.csa2_index_full(q, w, B.Rows(keys), torch.tensor([255], dtype=torch.int32, device=DEV), 256,
+                           scores=torch.zeros((1, 256), dtype=torch.int32, device=DEV))
+    assert int(st.item()) == 5       # SCORE_RANGE
+
+
+def test_index_bad_position_is_reported():
+    wl = synth.C0_TINY
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    bad = torch.tensor([5000], dtype=torch.int32, device=DEV)     # >= max_ctx
+    st = B.csa2_index_full(ly.q, ly.w, ly.keys, bad, c.max_ctx, P=16, pool_idx=ly.pool_idx[:, :16].contiguous(),
+                           pool_cnt=ly.pool_cnt)
+    assert int(st.item()) == 6
+    assert int(_np(ly.pool_cnt)[0]) == 0
+
+
+# ------------------------------------------------------------------ K2: top-k alone
+@pytest.mark.parametrize("n,k,spread", [(5000, 700, 3), (16384, 512, 50), (16385, 512, 50),
+                                        (70000, 16384, 1000), (70000, 300, 2), (300000, 16384, 10 ** 6)])
+def test_topk_pool_matches_oracle(n, k, spread):
+    rng = np.random.default_rng(n + k)
+    nq = 3
+    s = rng.integers(-spread, spread + 1, size=(nq, n)).astype(np.int32)
+    nv = np.array([n, n // 2 + 1, min(n, k // 2)], dtype=np.int32)
+    out = torch.empty((nq, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((nq,), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_topk_pool(torch.from_numpy(s).to(DEV), k, out, out_cnt=cnt,
+                                    n_valid=torch.from_numpy(nv).to(DEV)))
+    o, c = _np(out), _np(cnt)
+    for i in range(nq):
+        ref = O.top_k_positions(s[i, :nv[i]], np.arange(nv[i]), k)
+        assert c[i] == len(ref) and np.array_equal(o[i, :c[i]], ref)
+        assert (o[i, c[i]:] == -1).all()
+
+
+@pytest.mark.parametrize("n", [1000, 40000])
+def test_topk_all_equal_and_two_valued(n):
+    for s in (np.zeros((1, n), np.int32), np.where(np.arange(n) % 3 == 0, 7, -7).astype(np.int32)[None]):
+        k = 600
+        out = torch.empty((1, k), dtype=torch.int32, device=DEV)
+        B.check_status(B.csa2_topk_pool(torch.from_numpy(s).to(DEV), k, out))
+        assert np.array_equal(_np(out)[0], O.top_k_positions(s[0], np.arange(n), k))
+
+
+def test_topk_with_candidate_positions():
+    rng = np.random.default_rng(5)
+    for n in (9000, 30000):
+        pos = np.sort(rng.choice(10 ** 6, size=n, replace=False)).astype(np.int32)
+        s = rng.integers(0, 40, size=n).astype(np.int32)
+        out = torch.empty((1, 512), dtype=torch.int32, device=DEV)
+        B.check_status(B.csa2_topk_pool(torch.from_numpy(s[None]).to(DEV), 512, out,
+                                        cand_pos=torch.from_numpy(pos[None]).to(DEV)))
+        assert np.array_equal(_np(out)[0], O.top_k_positions(s, pos, 512))
+
+
+def test_topk_rejects_unsorted_candidates():
+    s = torch.zeros((1, 100), dtype=torch.int32, device=DEV)
+    pos = torch.arange(100, dtype=torch.int32, device=DEV).flip(0)[None].contiguous()
+    out = torch.empty((1, 10), dtype=torch.int32, device=DEV)
+    st = B.csa2_topk_pool(s, 10, out, cand_pos=pos)
+    assert int(st.item()) == 8
+
+
+# ------------------------------------------------------------------ K3 reindex
+@pytest.mark.parametrize("pool", [1024, 16384])
+def test_reindex_matches_oracle(pool):
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(40000,), modes=(synth.FULL, synth.REINDEX), pool=pool)
+    c = G.build(wl)
+    full, re = c.layers_dev
+    B.check_status(B.csa2_index_full(full.q, full.w, full.keys, c.pos_dev, c.max_ctx, P=pool,
+                                     pool_idx=full.pool_idx, pool_cnt=full.pool_cnt))
+    scores = torch.empty((1, pool), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_reindex(re.q, re.w, re.keys, full.pool_idx, full.pool_cnt, wl.topk, re.sel_idx,
+                                  sel_cnt=re.sel_cnt, scores=scores))
+    q0, w0 = c.host_q[(0, 0)]
+    _, ref_pool, _ = O.full_index(q0, w0, c.host_keys[(0, 0)], 39999, pool, wl.topk)
+    q1, w1 = c.host_q[(1, 0)]
+    ref_s, ref_sel = O.reindex(q1, w1, c.host_keys[(1, 0)], ref_pool, wl.topk)
+    assert np.array_equal(_np(full.pool_idx)[0], ref_pool)
+    assert np.array_equal(_np(scores)[0], ref_s)
+    assert np.array_equal(_np(re.sel_idx)[0], ref_sel) and int(_np(re.sel_cnt)[0]) == len(ref_sel)
+
+
+# ------------------------------------------------------------------ K4 attention
+@pytest.mark.parametrize("wl", [synth.C0_TINY, synth.scaled(synth.C1_SINGLE, seq_lens=(3001,))],
+                         ids=["hq8_d128", "hq64_d512"])
+def test_sparse_attention_matches_oracle(wl):
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    pos = int(c.query_pos[0])
+    q, w = c.host_q[(0, 0)]
+    _, _, sel = O.full_index(q, w, c.host_keys[(0, 0)], pos, wl.pool, wl.topk)
+    sel_pad = np.full((1, wl.topk), -1, np.int32)
+    sel_pad[0, :len(sel)] = sel
+    sel_d = torch.from_numpy(sel_pad).to(DEV)
+    cnt_d = torch.tensor([len(sel)], dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_sparse_attn_fp4(ly.q_attn, ly.codes, ly.scales, c.pos_dev, sel_d, ly.out,
+                                          sel_cnt=cnt_d, window=wl.window, lse=ly.lse))
+    S = O.attention_set(sel, pos, wl.window)
+    codes, scales = c.fp4_host[(0, 0)]
+    ref, ref_lse = O.sparse_attention(c.host_qa[(0, 0)], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
+    ok, err = G.tol_ok(_np(ly.out.float())[0], ref)
+    assert ok, f"max abs err {err}"
+    assert np.allclose(_np(ly.lse)[0], ref_lse, atol=1e-3, rtol=1e-4)
+
+
+def test_sparse_attention_window_only_and_overlap():
+    wl = synth.scaled(synth.C0_TINY, seq_lens=(700,))
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    codes, scales = c.fp4_host[(0, 0)]
+    cases = [np.zeros(0, np.int64), np.arange(600, 700), np.array([0, 5, 580, 650, 699])]
+    for sel in cases:
+        sel_pad = np.full((1, wl.topk), -1, np.int32)
+        sel_pad[0, :len(sel)] = sel
+        B.check_status(B.csa2_sparse_attn_fp4(ly.q_attn, ly.codes, ly.scales, c.pos_dev,
+                                              torch.from_numpy(sel_pad).to(DEV), ly.out,
+                                              sel_cnt=torch.tensor([len(sel)], dtype=torch.int32, device=DEV),
+                                              window=wl.window))
+        S = O.attention_set(sel, 699, wl.window)
+        ref, _ = O.sparse_attention(c.host_qa[(0, 0)], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
+        ok, err = G.tol_ok(_np(ly.out.float())[0], ref)
+        assert ok, f"max abs err {err}"
+
+
+# ------------------------------------------------------------------ the whole plan
+def _check_plan(c, n_check=None, need_rows_from_oracle=False):
+    wl = c.wl
+    plan = B.csa2_layer_plan(list(wl.modes), c.layers_dev, query_pos=c.pos_dev, seq_of_query=c.seq_dev,
+                             max_ctx=c.max_ctx, P=wl.pool, K=wl.topk, window=wl.window)
+    B.check_status(plan.status)
+    nq = len(c.query_pos)
+    worst = 0.0
+    for i in range(nq if n_check is None else n_check):
+        pos = int(c.query_pos[i])
+        res = O.decode_layer_plan(wl.modes, G.oracle_layers(c, i), pos, wl.pool, wl.topk, wl.window)
+        for l, (r, ly) in enumerate(zip(res, c.layers_dev)):
+            if r.pool_idx is not None:
+                n = int(_np(ly.pool_cnt)[i])
+                assert n == len(r.pool_idx) and np.array_equal(_np(ly.pool_idx)[i, :n], r.pool_idx)
+            n = int(_np(ly.sel_cnt)[i])
+            assert n == len(r.sel_idx) and np.array_equal(_np(ly.sel_idx)[i, :n], r.sel_idx), f"layer {l}"
+            ok, err = G.tol_ok(_np(ly.out[i].float()), r.out)
+            worst = max(worst, err)
+            assert ok, f"query {i} layer {l}: max abs err {err}"
+    return worst
+
+
+def test_plan_8_layers_reduced_context():
+    wl = synth.scaled(synth.C2_1M_PLAN, seq_lens=(50003,))
+    c = G.build(wl)
+    _check_plan(c)
+
+
+def test_plan_paged_ragged_batch():
+    wl = synth.scaled(synth.C3_RAGGED, ragged=(4, 2000, 30000), modes=(synth.FULL, synth.REUSE, synth.REINDEX))
+    c = G.build(wl)
+    _check_plan(c)
+
+
+def test_plan_tiny_config():
+    c = G.build(synth.C0_TINY)
+    _check_plan(c)
+
+
+def test_plan_repeat_is_deterministic():
+    wl = synth.scaled(synth.C2_1M_PLAN, seq_lens=(30000,), modes=(synth.FULL, synth.REINDEX, synth.REUSE))
+    c = G.build(wl)
+    plan = B.csa2_layer_plan(list(wl.modes), c.layers_dev, query_pos=c.pos_dev, max_ctx=c.max_ctx,
+                             P=wl.pool, K=wl.topk, window=wl.window)
+    first = [ly.out.clone() for ly in c.layers_dev]
+    for _ in range(3):
+        plan.run()
+    torch.cuda.synchronize()
+    for a, ly in zip(first, c.layers_dev):
+        assert torch.equal(a, ly.out)

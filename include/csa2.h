@@ -151,6 +151,31 @@ int32_t csa2_topk_pool(const int32_t* scores, int64_t ld, const int32_t* n_valid
                        void* ws, size_t ws_bytes, int32_t* status, void* stream);
 size_t csa2_topk_pool_workspace(int32_t nq, int32_t n_max, int32_t k);
 
+/* csa2_topk_pool_noalloc: csa2_topk_pool without a caller workspace.  The
+ * pages have no counterpart to this call; it exists for callers that cannot
+ * allocate device memory.  Plugin code inside a host framework may receive only
+ * its input and output buffers, and a serving loop may have reserved all
+ * device memory up front (cudaMalloc can block on the device and fragment
+ * that reservation).
+ * Arguments, results and errors are those of csa2_topk_pool, minus ws/ws_bytes.
+ * Scratch: one fixed device array inside the library, CSA2_NOALLOC_SCRATCH_BYTES
+ * long.  Every GPU that loads the library holds it until the process exits.
+ * n_max <= 16384 needs no scratch.  Larger sizes must satisfy
+ * csa2_topk_pool_workspace(nq, n_max, k) <= CSA2_NOALLOC_SCRATCH_BYTES;
+ * otherwise the call returns CSA2_ERR_WORKSPACE and launches nothing.  That
+ * allows 14 queries of up to 10^6 candidates each, or 13 of up to 2^24.
+ * The call allocates and frees nothing.  Its first call on a device looks up
+ * the array's address there (cudaGetSymbolAddress), so make that first call
+ * before any stream capture on that device.
+ * Every call uses the same array and clears the parts that must start at
+ * zero.  Calls that overlap on the GPU (other streams, other threads) race on
+ * it, so serialise them.
+ */
+#define CSA2_NOALLOC_SCRATCH_BYTES (4u << 20)
+int32_t csa2_topk_pool_noalloc(const int32_t* scores, int64_t ld, const int32_t* n_valid,
+                               const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
+                               int32_t* out_idx, int32_t* out_cnt, int32_t* status, void* stream);
+
 /* ------------------------------------------------------------ step 3
  * csa2_reindex: score only the pool positions with this layer's query,
  * weights and index keys, and keep the best K ("later layers search only that

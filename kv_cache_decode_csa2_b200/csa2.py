@@ -63,6 +63,7 @@ _SIGS = {
     "csa2_index_full_workspace": (_SZ, [_I32, _I32, _I32, _I32]),
     "csa2_topk_pool": (_I32, [_P, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
     "csa2_topk_pool_workspace": (_SZ, [_I32, _I32, _I32]),
+    "csa2_topk_pool_noalloc": (_I32, [_P, _I64, _P, _P, _I32, _I32, _I32, _P, _P, _P, _P]),
     "csa2_reindex": (_I32, [_P, _P, _RP, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _P, _P, _P, _P, _SZ,
                             _P, _P]),
     "csa2_reindex_workspace": (_SZ, [_I32, _I32, _I32]),

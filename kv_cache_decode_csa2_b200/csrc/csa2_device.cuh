@@ -221,23 +221,23 @@ __host__ __device__ __forceinline__ uint32_t swizzled_chunk(uint32_t r, uint32_t
 }
 
 // ------------------------------------------------------------------ scores
-// 12-bit bucket, non-decreasing in the score, used by the radix top-k.
-// Non-negative scores map to 2048 + f(s); negative ones to 2047 - f(-s-1).
-// f keeps the leading bit position and the 6 bits below it, so for s >= 64
-// a bucket spans 2^(e-6) consecutive scores, where e is the leading bit.
+// 13-bit bucket, non-decreasing in the score, used by the radix top-k.
+// Non-negative scores map to 4096 + f(s); negative ones to 4095 - f(-s-1).
+// f keeps the position of the leading bit and the 7 bits below it, so for
+// s >= 128 a bucket spans 2^(e-7) consecutive scores, where e is the leading bit.
 __host__ __device__ __forceinline__ uint32_t score_f(uint32_t s) {
-  if (s < 64u) return s;
+  if (s < 128u) return s;
 #ifdef __CUDA_ARCH__
   const uint32_t e = 31u - __clz(s);
 #else
   const uint32_t e = 31u - __builtin_clz(s);
 #endif
-  return (e - 5u) * 64u + ((s >> (e - 6u)) & 63u);
+  return (e - 6u) * 128u + ((s >> (e - 7u)) & 127u);
 }
 __host__ __device__ __forceinline__ uint32_t score_bucket(int32_t s) {
-  return s >= 0 ? 2048u + score_f((uint32_t)s) : 2047u - score_f((uint32_t)(-(s + 1)));
+  return s >= 0 ? 4096u + score_f((uint32_t)s) : 4095u - score_f((uint32_t)(-(s + 1)));
 }
-constexpr int kBuckets = 4096;
+constexpr int kBuckets = 8192;
 
 // Ordering key of a candidate: larger key = better (higher score, then lower
 // position).  All keys of distinct positions differ.

@@ -48,7 +48,8 @@ struct IndexCfg {
   static constexpr int kStages = (D == 128) ? 8 : 12;         // >= 96 KiB in flight per SM
 };
 
-__device__ __forceinline__ void named_sync_epi() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+constexpr int kEpiThreads = 256;   // 8 epilogue warps: two per TMEM lane quarter, one per half of the heads
+__device__ __forceinline__ void named_sync_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
@@ -59,12 +60,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 }
 
 template <int D, int N>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(64 + kEpiThreads, 1)
 index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) {
   using Cfg = IndexCfg<D>;
   constexpr int NST = Cfg::kStages;
   constexpr int TILE = Cfg::kTile;
-  constexpr uint32_t TMEM_COLS = (2 * N <= 32) ? 32 : (2 * N <= 64) ? 64 : (2 * N <= 128) ? 128 : 256;
+  // As many TMEM accumulator buffers as fit in the 512 columns (at most 8),
+  // so the MMA can run up to NBUF tiles ahead of the epilogue.
+  constexpr int NBUF = (512 / N) < 8 ? (512 / N) : 8;
+  constexpr uint32_t TMEM_COLS = NBUF * N <= 32 ? 32 : NBUF * N <= 64 ? 64 : NBUF * N <= 128 ? 128 : NBUF * N <= 256 ? 256 : 512;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -72,15 +76,15 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   uint8_t* bmat = stages + NST * TILE;
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(bmat + N * D);
   int32_t* w_s = reinterpret_cast<int32_t*>(hist_s + kBuckets);
-  int32_t* prefix = w_s + 128;                                   // [nq + 1]
+  int32_t* part_s = w_s + 128;                                   // [2][128] partial sums of heads N/2..N-1
+  int32_t* prefix = part_s + 256;                                // [nq + 1]
   uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + ((a.nq + 2) & ~1));
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
   uint64_t* tfull = bars + 2 * NST;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* bready = tempty + 2;
-  uint64_t* done = bready + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done + 1);
+  uint64_t* tempty = tfull + NBUF;
+  uint64_t* bready = tempty + NBUF;                              // the segment's B operand is in place
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bready + 2);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
   unsigned long long* bound_acc = reinterpret_cast<unsigned long long*>(tmem_slot + 2);
 
@@ -106,12 +110,12 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NBUF; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], 128);
+      mbar_init(&tempty[i], kEpiThreads / 32);   // one arrival per epilogue warp
     }
-    mbar_init(bready, 128);
-    mbar_init(done, 1);
+    mbar_init(bready, kEpiThreads / 32);
+    *bound_acc = 0ull;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -152,205 +156,231 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     q0 = l;
   }
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && lo < hi) {
-      prefetch_tensormap(&kmap);
-      const uint64_t pol = l2_policy_evict_first();
-      int q = q0, cur = -1;
-      int32_t pos_q = 0, seq = 0;
-      int64_t it = 0;
-      for (int64_t item = lo; item < hi; ++item, ++it) {
-        while (item >= prefix[q + 1]) ++q;
-        if (q != cur) {
-          cur = q;
-          pos_q = __ldg(a.query_pos + q);
-          seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
-        }
-        const int32_t tile = (int32_t)(item - prefix[q]);
-        const int st = (int)(it % NST);
-        const uint32_t ph = (uint32_t)((it / NST) & 1);
-        if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) break;
-        int64_t r[2];
-        uint32_t bytes = 0;
+  // The CTA's items are processed one query segment at a time.  Within a
+  // segment the producer, the MMA issuer and the epilogue run as a pipeline.
+  // Between segments the whole CTA synchronises, so the B operand (the
+  // query) and the histogram can be swapped without any hand-off protocol.
+  // `git` numbers the items of the CTA and drives every barrier phase.
+  const int et = tid - 64;                 // epilogue thread 0..255 (negative for warps 0-1)
+  const int half = et >> 7;                // which half of the heads this epilogue warp sums
+  const int quarter = warp & 3;            // TMEM lanes this warp may access
+  const int row = quarter * 32 + lane;     // key row of the tile this thread owns
+  constexpr int NH = N >= 64 ? N / 2 : N;  // heads per half (N <= 32: the first half takes all)
+  const bool active = N >= 64 || half == 0;
+  int64_t git = 0;
+  int seg_count = 0;   // segments done by this CTA (bready phase)
+  int q = q0;
+  for (int64_t s_lo = lo; s_lo < hi;) {
+    while (s_lo >= prefix[q + 1]) ++q;
+    const int64_t s_hi = hi < (int64_t)prefix[q + 1] ? hi : (int64_t)prefix[q + 1];
+    const int n_it = (int)(s_hi - s_lo);
+    const int32_t tile0 = (int32_t)(s_lo - prefix[q]);
+    const int32_t pos_q = __ldg(a.query_pos + q);
+
+    // ---- segment set-up (epilogue threads): B operand = q rows 0..H-1, zero
+    // rows up to N, K-major with the tile swizzle, and the head weights.  The
+    // producer does not wait for it (key tiles do not depend on the query);
+    // the MMA issuer waits on `bready`.  The int32 overflow guard
+    // 128 * sum_h |w_h| * sum_d |q_hd| < 2^31 is checked off the critical path.
+    const int8_t* qsrc = a.q + (int64_t)q * a.H * D;
+    if (warp >= 2) {
+      for (int idx = et; idx < N * (D / 16); idx += kEpiThreads) {
+        const int r = idx / (D / 16), c = idx % (D / 16);
+        int4 v = make_int4(0, 0, 0, 0);
+        if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
+        *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
+      }
+      if (et < N) w_s[et] = et < a.H ? (int32_t)__ldg(a.w + (int64_t)q * a.H + et) : 0;
+      fence_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bready);
+      named_sync_epi();
+      if (et < a.H) {
+        int32_t sq = 0;
+        const int4* src = reinterpret_cast<const int4*>(qsrc + et * D);
+        for (int c = 0; c < D / 16; ++c) {
+          const int4 v = __ldg(src + c);
+          const int32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int32_t p0 = tile * 128 + 64 * j;
-          r[j] = -1;
-          if (p0 <= pos_q) {
-            r[j] = map_row(a.rows, seq, p0);
-            if (r[j] < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
-            else bytes += 64 * D;
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int b = 0; b < 4; ++b) sq += abs((int32_t)(int8_t)(wv[j] >> (8 * b)));
+        }
+        const unsigned long long t = (unsigned long long)sq * (unsigned long long)abs(w_s[et]);
+        if (t) atomicAdd(bound_acc, t);
+      }
+    }
+
+    if (warp == 0) {
+      // ---------------------------------------------------------- producer
+      if (lane == 0) {
+        prefetch_tensormap(&kmap);
+        const uint64_t pol = l2_policy_evict_first();
+        const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
+        int i = 0;
+        for (; i < n_it; ++i) {
+          const int64_t g = git + i;
+          const int st = (int)(g % NST);
+          const uint32_t ph = (uint32_t)((g / NST) & 1);
+          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) break;
+          const int32_t tile = tile0 + i;
+          int64_t r[2];
+          uint32_t bytes = 0;
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int32_t p0 = tile * 128 + 64 * j;
+            r[j] = -1;
+            if (p0 <= pos_q) {
+              r[j] = map_row(a.rows, seq, p0);
+              if (r[j] < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+              else bytes += 64 * D;
+            }
+          }
+          mbar_arrive_expect_tx(&full[st], bytes);
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            if (r[j] >= 0)
+              tma_load_2d(stages + st * TILE + j * 64 * D, &kmap, 0, (int32_t)r[j], &full[st], pol);
+        }
+        if (*abort_flag) {   // let loads already in flight land before moving on
+          const int64_t issued = git + i;
+          const int64_t n = i < NST ? i : NST;
+          for (int64_t k = issued - n; k < issued; ++k)
+            mbar_wait_drain(&full[k % NST], (uint32_t)((k / NST) & 1));
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------------------------------------------------- MMA issuer
+      if (lane == 0) {
+        constexpr uint32_t idesc = idesc_i8(128, N);
+        const uint32_t b_addr = smem_u32(bmat);
+        const bool bok = mbar_wait(bready, (uint32_t)(seg_count & 1), abort_flag);
+        tc_fence_after();
+        for (int i = 0; i < n_it && bok; ++i) {
+          const int64_t g = git + i;
+          const int st = (int)(g % NST);
+          const uint32_t ph = (uint32_t)((g / NST) & 1);
+          const int buf = (int)(g % NBUF);
+          const uint32_t tph = (uint32_t)((g / NBUF) & 1);
+          if (!mbar_wait(&full[st], ph, abort_flag)) break;
+          if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(stages + st * TILE);
+#pragma unroll
+          for (int k = 0; k < D / 32; ++k)
+            mma_i8(tmem_base + buf * N, smem_desc_kmajor(a_addr + 32 * k, D),
+                   smem_desc_kmajor(b_addr + 32 * k, D), idesc, k > 0 ? 1u : 0u);
+          mma_commit(&empty[st]);
+          mma_commit(&tfull[buf]);
+        }
+      }
+    } else {
+      // ---------------------------------------------------------- epilogue
+      // Two warps share each TMEM lane quarter: warps 2-5 sum heads [0, NH)
+      // and warps 6-9 heads [NH, N) of the same 128 key rows; the second
+      // group hands its partial sums over through a double-buffered shared
+      // array.  The TMEM load of tile i+1 is issued before the arithmetic of
+      // tile i, so its latency is hidden.  Every epilogue thread walks the same
+      // tiles and reaches the same named barriers even after a timeout (it
+      // then skips the TMEM reads and the stores).
+      constexpr bool kRegW = NH <= 32;       // 64 heads per half: weights stay in shared memory
+      int32_t wreg[kRegW ? NH : 1];
+      if constexpr (kRegW) {
+#pragma unroll
+        for (int h = 0; h < NH; ++h) wreg[h] = active ? w_s[half * NH + h] : 0;
+      }
+      const int32_t* wsh = w_s + half * NH;
+      auto taddr_of = [&](int64_t g) {
+        return tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((g % NBUF) * N + (active ? half * NH : 0));
+      };
+      auto wait_tile = [&](int64_t g) {
+        return __all_sync(0xffffffffu, mbar_wait(&tfull[g % NBUF], (uint32_t)((g / NBUF) & 1), abort_flag));
+      };
+      auto load = [&](uint32_t (&r)[NH], int64_t g) {
+        if constexpr (NH == 16) {
+          tmem_ld16(taddr_of(g), r);
+        } else {
+#pragma unroll
+          for (int c = 0; c < NH / 32; ++c)
+            tmem_ld32(taddr_of(g) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+        }
+      };
+      // one tile: `cur` holds its accumulators; prefetch the next tile into `nxt`
+      auto step = [&](uint32_t (&cur)[NH], bool okc, uint32_t (&nxt)[NH], bool& okn, int i) {
+        const int64_t g = git + i;
+        const bool has_next = i + 1 < n_it;
+        if (has_next) {
+          okn = wait_tile(g + 1);
+          if (okn) {
+            tc_fence_after();
+            load(nxt, g + 1);
           }
         }
-        mbar_arrive_expect_tx(&full[st], bytes);
+        int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent chains, no long serial sum
 #pragma unroll
-        for (int j = 0; j < 2; ++j)
-          if (r[j] >= 0)
-            tma_load_2d(stages + st * TILE + j * 64 * D, &kmap, 0, (int32_t)r[j], &full[st], pol);
-      }
-      if (*abort_flag) {   // let loads already in flight land before the CTA exits
-        const int64_t n = it < NST ? it : NST;
-        for (int64_t k = it - n; k < it; ++k) mbar_wait_drain(&full[k % NST], (uint32_t)((k / NST) & 1));
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, N);
-      const uint32_t b_addr = smem_u32(bmat);
-      int q = q0, cur = -1, seg = -1;
-      int64_t it = 0;
-      for (int64_t item = lo; item < hi; ++item, ++it) {
-        while (item >= prefix[q + 1]) ++q;
-        if (q != cur) {
-          cur = q;
-          ++seg;
-          if (!mbar_wait(bready, (uint32_t)(seg & 1), abort_flag)) break;
+        for (int h = 0; h < NH; ++h) part[h & 7] += (kRegW ? wreg[h] : wsh[h]) * max((int32_t)cur[h], 0);
+        int32_t s = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+        if (!active) s = 0;
+        if (half == 1) part_s[(g & 1) * 128 + row] = s;
+        named_sync_epi();
+        if (half == 0 && okc) {
+          s += part_s[(g & 1) * 128 + row];
+          const int32_t pos = (tile0 + i) * 128 + row;
+          if (pos <= pos_q) {
+            a.scores[(int64_t)q * a.ld + pos] = s;
+            atomicAdd(&hist_s[score_bucket(s)], 1u);
+          }
+        }
+        if (has_next) {
+          if (okn) tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[(g + 1) % NBUF]);
+        }
+      };
+      uint32_t ra[NH], rb[NH];
+      bool oka = false, okb = false;
+      if (n_it > 0) {
+        oka = wait_tile(git);
+        if (oka) {
           tc_fence_after();
+          load(ra, git);
+          tmem_wait_ld();
         }
-        const int st = (int)(it % NST);
-        const uint32_t ph = (uint32_t)((it / NST) & 1);
-        const int buf = (int)(it & 1);
-        const uint32_t tph = (uint32_t)((it >> 1) & 1);
-        if (!mbar_wait(&full[st], ph, abort_flag)) break;
-        if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t a_addr = smem_u32(stages + st * TILE);
-#pragma unroll
-        for (int k = 0; k < D / 32; ++k) {
-          mma_i8(tmem_base + buf * N, smem_desc_kmajor(a_addr + 32 * k, D),
-                 smem_desc_kmajor(b_addr + 32 * k, D), idesc, k > 0 ? 1u : 0u);
-        }
-        mma_commit(&empty[st]);
-        mma_commit(&tfull[buf]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[git % NBUF]);
       }
-      mma_commit(done);
-    }
-  } else {
-    // ------------------------------------------------------------ epilogue
-    // Every epilogue thread walks the same items and reaches the same named
-    // barriers even after a timeout (it then only skips the TMEM reads and the
-    // stores), so a failed wait can never strand the others at a barrier.
-    const int et = tid - 64;                 // 0..127
-    const int quarter = warp & 3;            // TMEM lanes this warp may access
-    const int row = quarter * 32 + lane;     // key row of the tile this thread owns
-    constexpr bool kRegW = N <= 64;
-    int32_t wreg[kRegW ? N : 1];
-    int q = q0, cur = -1;
-    int32_t pos_q = 0;
-    int64_t it = 0;
-    auto flush = [&](int qq) {
+      for (int i = 0; i < n_it; i += 2) {
+        step(ra, oka, rb, okb, i);
+        if (i + 1 < n_it) step(rb, okb, ra, oka, i + 1);
+      }
+      // this query's histogram goes to global memory
       named_sync_epi();
       if (a.hist) {
-        for (int b = et; b < kBuckets; b += 128) {
+        for (int b = et; b < kBuckets; b += kEpiThreads) {
           const uint32_t v = hist_s[b];
           if (v) {
-            atomicAdd(a.hist + (int64_t)qq * kBuckets + b, v);
+            atomicAdd(a.hist + (int64_t)q * kBuckets + b, v);
             hist_s[b] = 0;
           }
         }
       }
-      named_sync_epi();
-    };
-    for (int64_t item = lo; item < hi; ++item, ++it) {
-      while (item >= prefix[q + 1]) ++q;
-      if (q != cur) {
-        if (cur >= 0) flush(cur);
-        cur = q;
-        pos_q = __ldg(a.query_pos + q);
-        // B operand: q rows 0..H-1 (zero rows up to N), K-major with the tile swizzle.
-        const int8_t* qsrc = a.q + (int64_t)q * a.H * D;
-        for (int idx = et; idx < N * (D / 16); idx += 128) {
-          const int r = idx / (D / 16), c = idx % (D / 16);
-          int4 v = make_int4(0, 0, 0, 0);
-          if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
-          *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
-        }
-        if (et < N) w_s[et] = et < a.H ? (int32_t)__ldg(a.w + (int64_t)q * a.H + et) : 0;
-        if (et == 0) *bound_acc = 0ull;
-        fence_async_smem();
-        named_sync_epi();
-        // Overflow guard: 128 * sum_h |w_h| * sum_d |q_hd| must stay below 2^31.
-        if (et < a.H) {
-          int32_t sq = 0;
-          const int4* src = reinterpret_cast<const int4*>(qsrc + et * D);
-          for (int c = 0; c < D / 16; ++c) {
-            const int4 v = __ldg(src + c);
-            const int32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-#pragma unroll
-              for (int b = 0; b < 4; ++b) sq += abs((int32_t)(int8_t)(wv[j] >> (8 * b)));
-          }
-          atomicAdd(bound_acc, (unsigned long long)sq * (unsigned long long)abs(w_s[et]));
-        }
-        if constexpr (kRegW) {
-#pragma unroll
-          for (int h = 0; h < N; ++h) wreg[h] = w_s[h];
-        }
-        named_sync_epi();
-        if (et == 0 && (*bound_acc) * 128ull >= (1ull << 31)) record_error(a.status, CSA2_ERR_SCORE_RANGE);
-        mbar_arrive(bready);
-      }
-      const int32_t tile = (int32_t)(item - prefix[q]);
-      const int buf = (int)(it & 1);
-      const uint32_t tph = (uint32_t)((it >> 1) & 1);
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[buf], tph, abort_flag));
-      if (!ok) {
-        mbar_arrive(&tempty[buf]);
-        continue;
-      }
-      tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * N);
-      int32_t s = 0;
-      if constexpr (N == 16) {
-        uint32_t r16[16];
-        tmem_ld16(taddr, r16);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&tempty[buf]);
-#pragma unroll
-        for (int h = 0; h < 16; ++h) s += wreg[h] * max((int32_t)r16[h], 0);
-      } else if constexpr (kRegW) {
-        uint32_t r32[N / 32][32];
-#pragma unroll
-        for (int g = 0; g < N / 32; ++g) tmem_ld32(taddr + 32 * g, r32[g]);
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&tempty[buf]);
-#pragma unroll
-        for (int g = 0; g < N / 32; ++g)
-#pragma unroll
-          for (int h = 0; h < 32; ++h) s += wreg[g * 32 + h] * max((int32_t)r32[g][h], 0);
-      } else {
-#pragma unroll 1
-        for (int g = 0; g < N / 32; ++g) {
-          uint32_t r32[32];
-          tmem_ld32(taddr + 32 * g, r32);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < 32; ++h) s += w_s[g * 32 + h] * max((int32_t)r32[h], 0);
-        }
-        tc_fence_before();
-        mbar_arrive(&tempty[buf]);
-      }
-      const int32_t pos = tile * 128 + row;
-      if (pos <= pos_q) {
-        a.scores[(int64_t)q * a.ld + pos] = s;
-        atomicAdd(&hist_s[score_bucket(s)], 1u);
-      }
     }
-    if (cur >= 0) flush(cur);
+    tc_fence_before();
+    __syncthreads();   // the segment is done everywhere: B and the histogram may be reused
+    tc_fence_after();
+    if (tid == 64) {
+      if ((*bound_acc) * 128ull >= (1ull << 31)) record_error(a.status, CSA2_ERR_SCORE_RANGE);
+      *bound_acc = 0ull;
+    }
+    __syncthreads();
+    git += n_it;
+    ++seg_count;
+    s_lo = s_hi;
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    if (lo < hi) mbar_wait_drain(done, 0);
-    tmem_dealloc(tmem_base, TMEM_COLS);
-  }
+  if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
   if (tid == 0 && *abort_flag) record_error(a.status, CSA2_ERR_TIMEOUT);
 }
 
@@ -374,8 +404,8 @@ EncodeTiledFn encode_fn() {
 template <int D>
 size_t index_smem_bytes(int N, int nq) {
   using Cfg = IndexCfg<D>;
-  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)N * D + kBuckets * 4 + 128 * 4 +
-         (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 6) * 8 + 32;
+  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)N * D + kBuckets * 4 + 128 * 4 + 256 * 4 +
+         (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 + 32;
 }
 
 template <int D, int N>
@@ -384,7 +414,7 @@ cudaError_t launch_one(const CUtensorMap& map, const IndexArgs& a, int grid, cud
   static unsigned long long done = 0;
   cudaError_t e = ensure_smem(index_score_kernel<D, N>, (int)index_smem_bytes<D>(N, kMaxQueries), done);
   if (e != cudaSuccess) return e;
-  index_score_kernel<D, N><<<grid, 192, smem, st>>>(map, a);
+  index_score_kernel<D, N><<<grid, 64 + kEpiThreads, smem, st>>>(map, a);
   return cudaGetLastError();
 }
 

@@ -26,8 +26,8 @@ struct Carver {
 // Radix top-k scratch for nq queries and up to two thresholds per query.
 struct TopkScratch {
   uint32_t* hist;        // [nq][kBuckets]                 (zeroed before the histogram pass)
-  uint32_t* chunk_cnt;   // [nq][2][n_chunks]              members per chunk
-  uint64_t* cand;        // [nq][2][cand_cap]              threshold-bucket candidates
+  uint32_t* chunk_cnt;   // [nq][2][n_chunks] x 64 bit     published chunk counts (flag, count)
+  uint64_t* cand;        // [nq][2][cand_cap]              keys with bucket >= b*, in position order
   uint32_t* cand_cnt;    // [nq][2]
   uint64_t* kth;         // [nq][2]                        key of the k-th best candidate
   int32_t* thresh;       // [nq][2][2]                     bucket b*, members above b*
@@ -35,7 +35,7 @@ struct TopkScratch {
   int32_t cand_cap;
 };
 constexpr int kChunk = 4096;          // positions per chunk in the multi-CTA passes
-constexpr int kCandCap = 16384;       // threshold-bucket candidates kept per (query, k)
+constexpr int kCandCap = 24576;       // ordered candidates (bucket >= b*) kept per (query, k)
 
 size_t topk_scratch_bytes(int32_t nq, int32_t n_max);
 TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);

@@ -17,6 +17,7 @@
 // Several layers of a plan go into one launch (a job array), so independent
 // layers run side by side.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "csa2_device.cuh"
 #include "internal.h"
@@ -26,6 +27,7 @@ namespace csa2 {
 namespace {
 
 constexpr int kRows = 64;        // rows of S per CTA
+constexpr int kSelCache = 1024;  // selection entries kept in shared memory per CTA
 constexpr int kMaxJobs = kMaxAttnJobs;
 
 struct AttnJob {
@@ -53,19 +55,35 @@ struct AttnArgs {
   int32_t* status;
 };
 
-__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-  const uint32_t e = (b >> 3) & 15u, m = b & 7u;
-  float v = (e == 0) ? (float)m * 0.001953125f                                   // m * 2^-9
-                     : __int_as_float((int)(((e + 120u) << 23) | (m << 20)));   // 2^(e-7) * (1 + m/8)
-  if (e == 15u && m == 7u) v = __int_as_float(0x7fc00000);
-  return (b & 0x80u) ? -v : v;
+// Two E2M1 codes (low nibble = first element) -> f16x2, exactly (every E2M1
+// value is an f16 value).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}" : "=r"(r) : "r"(byte));
+  return r;
 }
-
-__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
-  // magnitudes of codes 0..7: 0, .5, 1, 1.5, 2, 3, 4, 6
-  const uint32_t e = (c >> 1) & 3u, m = c & 1u;
-  const float mag = (e == 0) ? 0.5f * (float)m : __int_as_float((int)(((e + 126u) << 23) | (m << 22)));
-  return (c & 8u) ? -mag : mag;
+// One E4M3 byte -> the f16x2 pair (s, s), exactly (E4M3 spans 2^-9..448).
+__device__ __forceinline__ uint32_t e4m3_to_f16x2_pair(uint32_t byte) {
+  uint32_t r;
+  const uint16_t two = (uint16_t)(byte | (byte << 8));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(two));
+  return r;
+}
+// Four packed codes (8 elements) times their block scale -> 4 bf16x2 words.
+// The f16 product is exact (at most 6 significant bits, between 2^-10 and
+// 2688), and so is its bf16 copy.
+__device__ __forceinline__ void dequant8(uint32_t codes, uint32_t scale_byte, uint32_t (&out)[4]) {
+  const __half2 s2 = __halves2half2(__ushort_as_half((uint16_t)(e4m3_to_f16x2_pair(scale_byte) & 0xFFFFu)),
+                                    __ushort_as_half((uint16_t)(e4m3_to_f16x2_pair(scale_byte) & 0xFFFFu)));
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t h = e2m1x2_to_f16x2((codes >> (8 * e)) & 0xFFu);
+    __half2 v = *reinterpret_cast<const __half2*>(&h);
+    v = __hmul2(v, s2);
+    const float2 f = __half22float2(v);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(f.x, f.y);
+    out[e] = *reinterpret_cast<const uint32_t*>(&b);
+  }
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -100,7 +118,9 @@ struct AttnSmem {
   static constexpr size_t so = po + (size_t)HG * kP;
   static constexpr size_t mo = so + (size_t)HG * kS * 4;
   static constexpr size_t pos_o = mo + (size_t)HG * 8;
-  static constexpr size_t total = pos_o + kRows * 4 + 64;
+  static constexpr size_t row_o = pos_o + kRows * 4;
+  static constexpr size_t sel_o = row_o + 2 * kRows * 8;
+  static constexpr size_t total = sel_o + kSelCache * 4 + 64;
 };
 
 template <int D, int HG>
@@ -118,6 +138,8 @@ __global__ void __launch_bounds__(256, 1) sparse_attn_kernel(const __grid_consta
   float* s_s = reinterpret_cast<float*>(sm + L::so);
   float* ml_s = reinterpret_cast<float*>(sm + L::mo);     // [HG][2]: running max (log2 units), sum
   int32_t* pos_s = reinterpret_cast<int32_t*>(sm + L::pos_o);
+  int64_t* row_s = reinterpret_cast<int64_t*>(sm + L::row_o);     // [2][kRows]: code row, scale row
+  int32_t* sel_s = reinterpret_cast<int32_t*>(sm + L::sel_o);     // first kSelCache selection entries
   __shared__ int32_t meta[4];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -126,25 +148,56 @@ __global__ void __launch_bounds__(256, 1) sparse_attn_kernel(const __grid_consta
   const AttnJob& J = a.jobs[job_i];
   const int h0 = hg * HG;
 
-  if (tid == 0) {
-    const int32_t pos = __ldg(a.query_pos + q);
-    int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
-    cnt = cnt < 0 ? 0 : (cnt > a.K ? a.K : cnt);
-    const int32_t ws = pos - a.window + 1 > 0 ? pos - a.window + 1 : 0;
-    int l = 0, r = cnt;   // selection entries below the window start
-    const int32_t* sel = J.sel_idx + (int64_t)q * a.K;
-    while (l < r) {
-      const int m = (l + r) >> 1;
-      if (__ldg(sel + m) < ws) l = m + 1; else r = m;
-    }
-    meta[0] = pos;
-    meta[1] = ws;
-    meta[2] = l;                             // selection rows before the window
-    meta[3] = pos >= 0 ? l + (pos - ws + 1) : 0;   // |S|
-    if (pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+  // ---- Every load that does not depend on another is issued first: the Q
+  // rows of this head group, the query position and the selection count.
+  constexpr int QPER = HG * (D / 8) / 256;
+  int4 qv[QPER];
+#pragma unroll
+  for (int i = 0; i < QPER; ++i) {
+    const int idx = tid + i * 256, h = idx / (D / 8), c = idx % (D / 8);
+    qv[i] = h0 + h < a.Hq ? __ldg(reinterpret_cast<const int4*>(J.q + ((size_t)q * a.Hq + h0 + h) * D) + c)
+                          : make_int4(0, 0, 0, 0);
   }
+  const int32_t pos = __ldg(a.query_pos + q);
+  int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
+  if (tid == 0) meta[2] = 0;
+#pragma unroll
+  for (int i = 0; i < QPER; ++i) {
+    const int idx = tid + i * 256, h = idx / (D / 8), c = idx % (D / 8);
+    *reinterpret_cast<int4*>(q_s + h * L::kQ + c * 16) = qv[i];
+  }
+  // ---- S = (selection entries below the window start) followed by the window.
+  // The selection is ascending, so those entries are a prefix of it.  Count
+  // them in parallel, keeping the first kSelCache entries in shared memory
+  // for the row positions below.
+  cnt = cnt < 0 ? 0 : (cnt > a.K ? a.K : cnt);
+  const int32_t wstart = pos - a.window + 1 > 0 ? pos - a.window + 1 : 0;
   __syncthreads();
-  const int32_t pos = meta[0], wstart = meta[1], nsel = meta[2], nS = meta[3];
+  {
+    const int32_t* sel = J.sel_idx + (int64_t)q * a.K;
+    int32_t below = 0;
+    for (int base = 0; base < cnt; base += 4 * 256) {
+      int32_t v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * 256 + tid;
+        v[u] = i < cnt ? __ldg(sel + i) : 0x7fffffff;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = base + u * 256 + tid;
+        below += v[u] < wstart;
+        if (i < kSelCache) sel_s[i] = v[u];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
+    if (lane == 0 && below) atomicAdd(&meta[2], below);
+  }
+  if (tid == 0 && pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+  __syncthreads();
+  const int32_t nsel = meta[2];
+  const int32_t nS = pos >= 0 ? nsel + (pos - wstart + 1) : 0;
   const int32_t r0 = chunk * kRows;
   const int nrows = nS - r0 < kRows ? nS - r0 : kRows;
   const size_t pidx = ((size_t)q * a.Hq) * a.n_chunks + chunk;   // + h * n_chunks
@@ -158,56 +211,54 @@ __global__ void __launch_bounds__(256, 1) sparse_attn_kernel(const __grid_consta
   }
   const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
 
-  // ---- positions of this chunk's rows
+  // ---- positions and physical rows of this chunk's rows
   if (tid < kRows) {
     int32_t p = -1;
+    int64_t cr = -1, sr = -1;
     const int j = r0 + tid;
     if (tid < nrows) {
-      p = j < nsel ? __ldg(J.sel_idx + (int64_t)q * a.K + j) : wstart + (j - nsel);
+      p = j < nsel ? (j < kSelCache ? sel_s[j] : __ldg(J.sel_idx + (int64_t)q * a.K + j)) : wstart + (j - nsel);
       if (p < 0 || p > pos) {
         record_error(a.status, CSA2_ERR_INDEX_RANGE);
         p = -1;
       }
     }
-    pos_s[tid] = p;
-  }
-  // ---- Q rows of this head group
-  for (int i = tid; i < HG * (D / 8); i += blockDim.x) {
-    const int h = i / (D / 8), c = i % (D / 8);
-    int4 v = make_int4(0, 0, 0, 0);
-    if (h0 + h < a.Hq) v = __ldg(reinterpret_cast<const int4*>(J.q + ((size_t)q * a.Hq + h0 + h) * D) + c);
-    *reinterpret_cast<int4*>(q_s + h * L::kQ + c * 16) = v;
-  }
-  __syncthreads();
-  // ---- gather + dequantise: one (row, 32-element block) per item
-  for (int i = tid; i < kRows * (D / 32); i += blockDim.x) {
-    const int r = i / (D / 32), blk = i % (D / 32);
-    const int32_t p = pos_s[r];
-    uint4 codes = make_uint4(0, 0, 0, 0);
-    float sc = 0.f;
     if (p >= 0) {
-      const int64_t cr = map_row(J.cmap, seq, p), sr = map_row(J.smap, seq, p);
+      cr = map_row(J.cmap, seq, p);
+      sr = map_row(J.smap, seq, p);
       if (cr < 0 || sr < 0) {
         record_error(a.status, CSA2_ERR_INDEX_RANGE);
-      } else {
-        codes = __ldg(reinterpret_cast<const uint4*>(J.codes + cr * J.codes_rb) + blk);
-        sc = e4m3_to_float(__ldg(J.scales + sr * J.scales_rb + blk));
+        p = -1;
+        cr = sr = -1;
       }
     }
-    const uint32_t cw[4] = {codes.x, codes.y, codes.z, codes.w};
-    uint32_t packed[16];
+    pos_s[tid] = p;
+    row_s[tid] = cr;
+    row_s[kRows + tid] = sr;
+  }
+  __syncthreads();
+  // ---- gather + dequantise: one (row, 8-element group) per item, so a warp
+  // reads 128 consecutive code bytes of a row and writes 512 consecutive bytes
+  // of shared memory (no bank conflicts).  All code words and scales of a
+  // thread are loaded before any is used.
+  {
+    constexpr int DPER = kRows * (D / 8) / 256;
+    uint32_t cw[DPER];
+    uint32_t sb[DPER];
 #pragma unroll
-    for (int wv = 0; wv < 4; ++wv)
+    for (int u = 0; u < DPER; ++u) {
+      const int i = tid + u * 256, r = i / (D / 8), g = i % (D / 8);
+      const int64_t cr = row_s[r], sr = row_s[kRows + r];
+      cw[u] = cr >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(J.codes + cr * J.codes_rb) + g) : 0u;
+      sb[u] = cr >= 0 ? (uint32_t)__ldg(J.scales + sr * J.scales_rb + g / 4) : 0u;
+    }
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t byte = (cw[wv] >> (8 * e)) & 0xFFu;
-        const __nv_bfloat16 lo = __float2bfloat16_rn(e2m1_to_float(byte & 0xFu) * sc);
-        const __nv_bfloat16 hi = __float2bfloat16_rn(e2m1_to_float(byte >> 4) * sc);
-        packed[wv * 4 + e] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
-      }
-    uint4* dst = reinterpret_cast<uint4*>(kv_s + r * L::kKV + blk * 64);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) dst[k] = make_uint4(packed[4 * k], packed[4 * k + 1], packed[4 * k + 2], packed[4 * k + 3]);
+    for (int u = 0; u < DPER; ++u) {
+      const int i = tid + u * 256, r = i / (D / 8), g = i % (D / 8);
+      uint32_t packed[4];
+      dequant8(cw[u], sb[u], packed);
+      *reinterpret_cast<uint4*>(kv_s + r * L::kKV + g * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    }
   }
   __syncthreads();
 
@@ -316,27 +367,57 @@ __global__ void __launch_bounds__(256, 1) sparse_attn_kernel(const __grid_consta
 }
 
 // Merges the chunk partials of one (job, query, head): o = sum_c 2^(m_c-M) O_c / L.
+// Each thread owns 4 output columns; every chunk's (max, sum) and partial
+// columns are loaded up front so the loads overlap.
 template <int D>
 __global__ void __launch_bounds__(D / 4) attn_combine_kernel(const __grid_constant__ AttnArgs a) {
+  constexpr int kMaxChunks = 24;
   const int h = blockIdx.x;
   const int job_i = blockIdx.y / a.nq, q = blockIdx.y % a.nq;
   const AttnJob& J = a.jobs[job_i];
   const size_t base = ((size_t)q * a.Hq + h) * a.n_chunks;
+  const int d = threadIdx.x * 4;
   float M = -INFINITY;
-  for (int c = 0; c < a.n_chunks; ++c) M = fmaxf(M, J.part_ml[(base + c) * 2]);
   float Lsum = 0.f;
   float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int d = threadIdx.x * 4;
-  for (int c = 0; c < a.n_chunks; ++c) {
-    const float m = J.part_ml[(base + c) * 2];
-    if (m == -INFINITY) continue;
-    const float e = exp2f(m - M);
-    Lsum += e * J.part_ml[(base + c) * 2 + 1];
-    const float4 v = *reinterpret_cast<const float4*>(J.part_o + (base + c) * D + d);
-    o.x += e * v.x;
-    o.y += e * v.y;
-    o.z += e * v.z;
-    o.w += e * v.w;
+  if (a.n_chunks > kMaxChunks) {   // long selections: plain two-pass loop
+    for (int c = 0; c < a.n_chunks; ++c) M = fmaxf(M, J.part_ml[(base + c) * 2]);
+    for (int c = 0; c < a.n_chunks; ++c) {
+      const float mc = J.part_ml[(base + c) * 2];
+      if (mc == -INFINITY) continue;
+      const float e = exp2f(mc - M);
+      Lsum += e * J.part_ml[(base + c) * 2 + 1];
+      const float4 vc = *reinterpret_cast<const float4*>(J.part_o + (base + c) * D + d);
+      o.x += e * vc.x;
+      o.y += e * vc.y;
+      o.z += e * vc.z;
+      o.w += e * vc.w;
+    }
+  } else {
+  float m[kMaxChunks], l[kMaxChunks];
+  float4 v[kMaxChunks];
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (c < a.n_chunks) {
+      const float2 ml = *reinterpret_cast<const float2*>(J.part_ml + (base + c) * 2);
+      m[c] = ml.x;
+      l[c] = ml.y;
+      v[c] = ml.x == -INFINITY ? make_float4(0.f, 0.f, 0.f, 0.f)
+                               : *reinterpret_cast<const float4*>(J.part_o + (base + c) * D + d);
+      M = fmaxf(M, ml.x);
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < kMaxChunks; ++c) {
+    if (c < a.n_chunks && m[c] != -INFINITY) {
+      const float e = exp2f(m[c] - M);
+      Lsum += e * l[c];
+      o.x += e * v[c].x;
+      o.y += e * v[c].y;
+      o.z += e * v[c].z;
+      o.w += e * v[c].w;
+    }
+  }
   }
   const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
   uint16_t* dst = J.out + ((size_t)q * a.Hq + h) * D + d;

@@ -7,21 +7,26 @@
 // are distinct, and a larger key is a better candidate: higher score, then
 // lower index.  The index order equals the position order because candidate
 // positions ascend.  The top-k is therefore {j : key_j >= kth}, where kth
-// is the k-th largest key.  Finding kth is a radix select; writing the
-// members in index order is a stable stream compaction, so no sort is needed.
+// is the k-th largest key.
 //
-// Large n (multi-CTA, one chunk of kChunk candidates per CTA):
-//   hist    12-bit monotone score buckets -> per-query histogram (fused into
-//           the index-score kernel when the scores come from there)
-//   select  each CTA finds the threshold bucket b* from the histogram, counts
-//           its members above b*, and appends threshold-bucket keys to a
-//           candidate list
-//   resolve one CTA per (query, k): radix select of the k-th key among the
-//           threshold-bucket keys (in shared memory; a global-memory fallback
-//           covers lists that overflow), then per-chunk member counts
-//   write   each CTA writes its chunk's members at the prefix of the counts
-//           of the chunks before it
+// Every candidate also gets a 13-bit bucket, monotone in its score.  Counting
+// buckets gives the threshold bucket b*: everything above b* is in, and
+// the k-th key is among the b* candidates ("ties").  A radix select on the
+// ties finds it, and a stable compaction writes the members in position
+// order.  No sort is needed.
+//
+// Large n (multi-CTA):
+//   hist    bucket histogram (fused into the index-score kernel when the scores
+//           come from there)
+//   gather  one CTA per 4096-candidate chunk: finds b* from the histogram,
+//           counts the chunk's candidates with bucket >= b*, publishes the
+//           count, adds up the counts of the chunks before it (bounded wait),
+//           and writes those candidates' keys in position order
+//   finish  one CTA per (query, k): radix select of the k-th key among the
+//           ties of its ordered candidate list, then the ordered compaction
 // Small n (<= kSmallMax): one CTA per query does all of this in shared memory.
+// Bucket histograms use plain shared atomics (scores spread over many buckets);
+// the digit histograms of the radix select, where lanes collide, are warp-aggregated.
 #include "csa2_device.cuh"
 #include "internal.h"
 
@@ -39,7 +44,7 @@ TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max) {
   if (s.n_chunks < 1) s.n_chunks = 1;
   s.cand_cap = kCandCap;
   s.hist = c.take<uint32_t>((size_t)nq * kBuckets);
-  s.chunk_cnt = c.take<uint32_t>((size_t)nq * 2 * s.n_chunks);
+  s.chunk_cnt = c.take<uint32_t>((size_t)nq * 2 * s.n_chunks * 2);   // published (flag, count) pairs
   s.cand = c.take<uint64_t>((size_t)nq * 2 * s.cand_cap);
   s.cand_cnt = c.take<uint32_t>((size_t)nq * 2);
   s.kth = c.take<uint64_t>((size_t)nq * 2);
@@ -76,6 +81,16 @@ __device__ __forceinline__ int32_t pos_of(const CandView& v, int q, int32_t j) {
 }
 
 __device__ __forceinline__ uint64_t key_of(int32_t score, int32_t j) { return cand_key(score, j); }
+__device__ __forceinline__ int32_t key_index(uint64_t key) { return key_pos(key); }
+__device__ __forceinline__ int32_t key_bucket(uint64_t key) { return (int32_t)score_bucket(key_score(key)); }
+
+// One increment of hist[bin] per active lane, aggregated over lanes that hit
+// the same bin.  All 32 lanes of the warp must call it.
+__device__ __forceinline__ void agg_inc(uint32_t* hist, uint32_t bin, bool active) {
+  const uint32_t v = active ? bin : 0xFFFFFFFFu;
+  const uint32_t peers = __match_any_sync(0xffffffffu, v);
+  if (active && (threadIdx.x & 31) == (uint32_t)(__ffs(peers) - 1)) atomicAdd(hist + bin, (uint32_t)__popc(peers));
+}
 
 // Block-wide exclusive scan of one int per thread (blockDim.x <= 1024).
 __device__ __forceinline__ int32_t block_excl_scan(int32_t v, int32_t* tmp, int32_t* total) {
@@ -104,19 +119,33 @@ __device__ __forceinline__ int32_t block_excl_scan(int32_t v, int32_t* tmp, int3
   return base + x - v;
 }
 
-// Threshold bucket for k from a 4096-bucket histogram: the largest b with
-// count(>= b) >= k.  Returns b* (or -1 when every candidate is a member) and
-// the count strictly above it.  Called by all threads of a 256-thread block.
+// Threshold bucket for k: the largest b with count(>= b) >= k, or -1 when
+// there are at most k candidates (all are members).  Also returns the count
+// strictly above b*.  All NT threads of the block call it.  Each thread reads
+// its kBuckets/NT contiguous bins with 16-byte loads, all issued before any
+// is used (the histogram may be in global or shared memory).
+template <int NT>
 __device__ void find_threshold(const uint32_t* hist, int32_t k, int32_t* out_b, int32_t* out_above,
                                int32_t* tmp) {
-  const int t = threadIdx.x;              // 256 threads x 16 buckets, from the top
-  int32_t seg[16];
+  constexpr int PER = kBuckets / NT;
+  static_assert(PER % 4 == 0, "bins per thread must be a multiple of 4");
+  const int t = threadIdx.x;
+  // thread t owns bins [kBuckets - (t+1)*PER, kBuckets - t*PER): the highest first
+  const uint4* src = reinterpret_cast<const uint4*>(hist + kBuckets - (t + 1) * PER);
+  uint4 v[PER / 4];
+#pragma unroll
+  for (int i = 0; i < PER / 4; ++i) v[i] = src[i];
+  uint32_t bins[PER];
+#pragma unroll
+  for (int i = 0; i < PER / 4; ++i) {
+    bins[4 * i] = v[i].x;
+    bins[4 * i + 1] = v[i].y;
+    bins[4 * i + 2] = v[i].z;
+    bins[4 * i + 3] = v[i].w;
+  }
   int32_t sum = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    seg[i] = (int32_t)hist[kBuckets - 1 - (t * 16 + i)];
-    sum += seg[i];
-  }
+  for (int i = 0; i < PER; ++i) sum += (int32_t)bins[i];
   int32_t total;
   const int32_t before = block_excl_scan(sum, tmp, &total);   // count in higher segments
   if (t == 0 && total <= k) {
@@ -126,109 +155,25 @@ __device__ void find_threshold(const uint32_t* hist, int32_t k, int32_t* out_b, 
   if (total > k && before < k && before + sum >= k) {
     int32_t acc = before;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      if (acc + seg[i] >= k) {
-        *out_b = kBuckets - 1 - (t * 16 + i);
+    for (int i = PER - 1; i >= 0; --i) {     // from this thread's highest bin down
+      const int32_t c = (int32_t)bins[i];
+      if (acc + c >= k) {
+        *out_b = kBuckets - (t + 1) * PER + i;
         *out_above = acc;
         break;
       }
-      acc += seg[i];
+      acc += c;
     }
   }
   __syncthreads();
 }
 
-// ------------------------------------------------------------------ hist
-__global__ void __launch_bounds__(256) topk_hist_kernel(CandView v, uint32_t* hist) {
-  __shared__ uint32_t h[kBuckets];
-  const int q = blockIdx.y;
-  const int32_t n = n_of(v, q);
-  const int64_t j0 = (int64_t)blockIdx.x * kChunk;
-  if (j0 >= n) return;
-  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) h[i] = 0;
-  __syncthreads();
-  const int32_t j1 = (int32_t)(j0 + kChunk < (int64_t)n ? j0 + kChunk : (int64_t)n);
-  const int32_t* sc = v.scores + (int64_t)q * v.ld;
-  for (int32_t j = (int32_t)j0 + threadIdx.x; j < j1; j += blockDim.x)
-    atomicAdd(&h[score_bucket(__ldg(sc + j))], 1u);
-  __syncthreads();
-  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x)
-    if (h[i]) atomicAdd(hist + (int64_t)q * kBuckets + i, h[i]);
-}
-
-// ------------------------------------------------------------------ select
-struct SelectArgs {
-  CandView v;
-  TopkScratch s;
-  int32_t k[2];
-  int32_t n_k;
-  int32_t* status;
-};
-
-__global__ void __launch_bounds__(256) topk_select_kernel(SelectArgs a) {
-  __shared__ int32_t tmp[32];
-  __shared__ int32_t b_s[2], above_s[2];
-  __shared__ uint32_t cnt_s[2];
-  const int q = blockIdx.y, c = blockIdx.x;
-  const int32_t n = n_of(a.v, q);
-  const uint32_t* hist = a.s.hist + (int64_t)q * kBuckets;
-  for (int t = 0; t < a.n_k; ++t) find_threshold(hist, a.k[t], &b_s[t], &above_s[t], tmp);
-  if (threadIdx.x < 2) cnt_s[threadIdx.x] = 0;
-  if (c == 0 && threadIdx.x < a.n_k) {
-    a.s.thresh[(q * 2 + threadIdx.x) * 2 + 0] = b_s[threadIdx.x];
-    a.s.thresh[(q * 2 + threadIdx.x) * 2 + 1] = above_s[threadIdx.x];
-  }
-  __syncthreads();
-  const int64_t j0 = (int64_t)c * kChunk;
-  const int32_t j1 = (int32_t)(j0 + kChunk < (int64_t)n ? j0 + kChunk : (int64_t)n);
-  const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
-  const int lane = threadIdx.x & 31;
-  uint32_t mine[2] = {0, 0};
-  for (int64_t base = j0; base < j1; base += blockDim.x) {
-    const int32_t j = (int32_t)base + threadIdx.x;
-    const bool in = j < j1;
-    int32_t s = 0;
-    if (in) {
-      s = __ldg(sc + j);
-      if (a.v.cand_pos && j > 0 && j < n) {
-        if (pos_of(a.v, q, j) <= pos_of(a.v, q, j - 1)) record_error(a.status, CSA2_ERR_ORDER);
-      }
-    }
-    const int32_t b = in ? (int32_t)score_bucket(s) : -2;
-    for (int t = 0; t < a.n_k; ++t) {
-      if (b > b_s[t]) mine[t]++;
-      const bool tie = in && b == b_s[t];
-      const uint32_t m = __ballot_sync(0xffffffffu, tie);
-      if (m) {
-        uint32_t slot0 = 0;
-        const int leader = __ffs(m) - 1;
-        if (lane == leader) slot0 = atomicAdd(a.s.cand_cnt + q * 2 + t, (uint32_t)__popc(m));
-        slot0 = __shfl_sync(0xffffffffu, slot0, leader);
-        if (tie) {
-          const uint32_t slot = slot0 + __popc(m & ((1u << lane) - 1u));
-          if (slot < (uint32_t)a.s.cand_cap)
-            a.s.cand[((int64_t)q * 2 + t) * a.s.cand_cap + slot] = key_of(s, j);
-        }
-      }
-    }
-  }
-  for (int t = 0; t < a.n_k; ++t) {
-    uint32_t x = mine[t];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0 && x) atomicAdd(&cnt_s[t], x);
-  }
-  __syncthreads();
-  if (threadIdx.x < a.n_k)
-    a.s.chunk_cnt[((int64_t)q * 2 + threadIdx.x) * a.s.n_chunks + c] = cnt_s[threadIdx.x];
-}
-
-// ------------------------------------------------------------------ radix select
 // Returns, to every thread of the block, the need-th largest (1-based) of the
-// m distinct keys get(0..m-1).  The bits above the highest bit where the keys
-// differ are common (AND == OR there).  Digits of at most 8 bits are fixed
-// from there downwards.  The select stops early once every key under the fixed
-// prefix is a member: kth is then the smallest of those keys.
+// non-zero keys among get(0..m-1) (zero marks "not a candidate"; need is at
+// most the number of non-zero keys).  The bits above the highest bit where the
+// candidates differ are common; digits of at most 8 bits are fixed from there
+// downwards, and the select stops early once every key under the fixed prefix
+// is a member (kth is then the smallest of them).
 template <class Get>
 __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* hist256,
                                  unsigned long long* red) {
@@ -243,8 +188,10 @@ __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* his
   unsigned long long kand = ~0ull, kor = 0ull;
   for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
     const uint64_t k = get(i);
-    kand &= k;
-    kor |= k;
+    if (k) {
+      kand &= k;
+      kor |= k;
+    }
   }
   atomicAnd(&red[0], kand);
   atomicOr(&red[1], kor);
@@ -256,14 +203,16 @@ __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* his
   uint64_t fixed = (top == 63) ? 0ull : ~((2ull << top) - 1ull);   // bits above `top`
   uint64_t prefix = kand_all & fixed;
   int64_t r = need;
+  const int64_t m_pad = (m + 31) & ~int64_t(31);
   while (true) {
     const int lo = top >= 7 ? top - 7 : 0;
     const uint32_t dmask = (uint32_t)((2ull << (top - lo)) - 1ull);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) hist256[i] = 0;
     __syncthreads();
-    for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
-      const uint64_t k = get(i);
-      if ((k & fixed) == prefix) atomicAdd(&hist256[(uint32_t)(k >> lo) & dmask], 1u);
+    for (int64_t i = threadIdx.x; i < m_pad; i += blockDim.x) {
+      const uint64_t k = i < m ? get(i) : 0ull;
+      const bool in = k && (k & fixed) == prefix;
+      agg_inc(hist256, (uint32_t)(k >> lo) & dmask, in);
     }
     __syncthreads();
     if (threadIdx.x < 32) {   // walk digits from the top, 8 per lane
@@ -304,7 +253,7 @@ __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* his
       __syncthreads();
       for (int64_t i = threadIdx.x; i < m; i += blockDim.x) {
         const uint64_t k = get(i);
-        if ((k & fixed) == prefix) atomicMin(&red[0], (unsigned long long)k);
+        if (k && (k & fixed) == prefix) atomicMin(&red[0], (unsigned long long)k);
       }
       __syncthreads();
       const uint64_t res = red[0];
@@ -315,117 +264,289 @@ __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* his
   }
 }
 
-// ------------------------------------------------------------------ resolve
-struct ResolveArgs {
-  CandView v;
-  TopkScratch s;
-  int32_t k[2];
-};
-
-constexpr int kResolveSmemKeys = kCandCap;
-
-__global__ void __launch_bounds__(1024) topk_resolve_kernel(ResolveArgs a) {
-  extern __shared__ uint64_t keys_s[];
-  __shared__ uint32_t hist256[256];
-  __shared__ unsigned long long red[2];
-  const int q = blockIdx.x, t = blockIdx.y;
-  const int32_t n = n_of(a.v, q);
-  const int32_t k = a.k[t];
-  const int32_t bstar = a.s.thresh[(q * 2 + t) * 2 + 0];
-  const int32_t above = a.s.thresh[(q * 2 + t) * 2 + 1];
-  uint32_t* ccnt = a.s.chunk_cnt + ((int64_t)q * 2 + t) * a.s.n_chunks;
-  if (bstar < 0 || n <= k) {   // every candidate is a member
-    if (threadIdx.x == 0) a.s.kth[q * 2 + t] = 0ull;
-    return;
+// ------------------------------------------------------------------ hist
+__global__ void __launch_bounds__(256) topk_hist_kernel(CandView v, uint32_t* hist) {
+  __shared__ uint32_t h[kBuckets];
+  const int q = blockIdx.y;
+  const int32_t n = n_of(v, q);
+  const int32_t j0 = blockIdx.x * kChunk;
+  if (j0 >= n) return;
+  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) h[i] = 0;
+  __syncthreads();
+  const int32_t* sc = v.scores + (int64_t)q * v.ld;
+  constexpr int kPerT = kChunk / 256;
+  int32_t sr[kPerT];
+#pragma unroll
+  for (int i = 0; i < kPerT; ++i) {            // all loads in flight before any use
+    const int32_t j = j0 + i * 256 + threadIdx.x;
+    sr[i] = j < n ? __ldg(sc + j) : 0;
   }
-  const int64_t need = (int64_t)k - above;
-  const uint32_t m = a.s.cand_cnt[q * 2 + t];
-  uint64_t kth;
-  if (m <= (uint32_t)kResolveSmemKeys) {
-    const uint64_t* src = a.s.cand + ((int64_t)q * 2 + t) * a.s.cand_cap;
-    for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) keys_s[i] = src[i];
-    __syncthreads();
-    kth = radix_select([&](int64_t i) { return keys_s[i]; }, m, need, hist256, red);
-    for (uint32_t i = threadIdx.x; i < m; i += blockDim.x) {
-      const uint64_t key = keys_s[i];
-      if (key >= kth) atomicAdd(ccnt + (0xFFFFFFFFu - (uint32_t)key) / kChunk, 1u);
-    }
-  } else {
-    // Overflowed candidate list (a very flat score distribution): select over
-    // the whole score row, restricted to the threshold bucket.
-    const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
-    auto get = [&](int64_t j) -> uint64_t {
-      const int32_t s = __ldg(sc + j);
-      return (int32_t)score_bucket(s) == bstar ? key_of(s, (int32_t)j) : 0ull;
-    };
-    // Keys outside the bucket map to 0, below every real key (a real key has
-    // an index < 2^31 in its low half, so it is never 0).  need is at most the
-    // bucket's count, so the need-th largest is always a real key.
-    kth = radix_select(get, n, need, hist256, red);
-    for (int64_t j = threadIdx.x; j < n; j += blockDim.x) {
-      const uint64_t key = get(j);
-      if (key != 0ull && key >= kth) atomicAdd(ccnt + j / kChunk, 1u);
-    }
+#pragma unroll
+  for (int i = 0; i < kPerT; ++i) {
+    const int32_t j = j0 + i * 256 + threadIdx.x;
+    if (j < n) atomicAdd(&h[score_bucket(sr[i])], 1u);
   }
-  if (threadIdx.x == 0) a.s.kth[q * 2 + t] = kth;
+  __syncthreads();
+  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x)
+    if (h[i]) atomicAdd(hist + (int64_t)q * kBuckets + i, h[i]);
 }
 
-// ------------------------------------------------------------------ write
-struct WriteArgs {
-  CandView v;
+// ------------------------------------------------------------------ thresholds
+struct ThreshArgs {
   TopkScratch s;
-  TopkOut out[2];
+  int32_t k[2];
   int32_t n_k;
 };
 
-__global__ void __launch_bounds__(256) topk_write_kernel(WriteArgs a) {
+// One CTA per query: the threshold bucket and the count above it, per k.
+__global__ void __launch_bounds__(256) topk_thresh_kernel(ThreshArgs a) {
+  __shared__ int32_t tmp[32];
+  __shared__ int32_t b_s, above_s;
+  const int q = blockIdx.x;
+  const uint32_t* hist = a.s.hist + (int64_t)q * kBuckets;
+  for (int t = 0; t < a.n_k; ++t) {
+    find_threshold<256>(hist, a.k[t], &b_s, &above_s, tmp);
+    if (threadIdx.x == 0) {
+      a.s.thresh[(q * 2 + t) * 2 + 0] = b_s;
+      a.s.thresh[(q * 2 + t) * 2 + 1] = above_s;
+    }
+    __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ gather
+struct GatherArgs {
+  CandView v;
+  TopkScratch s;
+  int32_t n_k;
+  int32_t* status;
+};
+
+constexpr int kPer = kChunk / 256;   // candidates per thread in the chunk kernel
+
+__device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__global__ void __launch_bounds__(256) topk_gather_kernel(GatherArgs a) {
   __shared__ int32_t tmp[32];
   __shared__ int32_t base_s;
   const int q = blockIdx.y, c = blockIdx.x;
   const int32_t n = n_of(a.v, q);
-  const int32_t chunks_q = (int32_t)(((int64_t)n + kChunk - 1) / kChunk);
-  for (int t = 0; t < a.n_k; ++t) {
-    const TopkOut o = a.out[t];
-    const uint32_t* ccnt = a.s.chunk_cnt + ((int64_t)q * 2 + t) * a.s.n_chunks;
-    const uint64_t kth = a.s.kth[q * 2 + t];
-    int32_t* dst = o.idx + (int64_t)q * o.k;
-    const int32_t total = n < o.k ? n : o.k;
-    if (c == (chunks_q > 0 ? chunks_q - 1 : 0)) {
-      for (int32_t i = total + threadIdx.x; i < o.k; i += blockDim.x) dst[i] = -1;
-      if (threadIdx.x == 0 && o.cnt) o.cnt[q] = total;
+  const int32_t j0 = c * kChunk + threadIdx.x * kPer;
+  const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
+  int32_t s[kPer];
+  int32_t bk[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int32_t j = j0 + i;
+    s[i] = j < n ? __ldg(sc + j) : 0;
+  }
+  int32_t bst[2];
+  bst[0] = a.s.thresh[(q * 2 + 0) * 2];
+  bst[1] = a.n_k > 1 ? a.s.thresh[(q * 2 + 1) * 2] : 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) bk[i] = j0 + i < n ? (int32_t)score_bucket(s[i]) : -2;
+  if (a.v.cand_pos) {
+    int32_t p[kPer + 1];
+#pragma unroll
+    for (int i = 0; i <= kPer; ++i) {
+      const int32_t j = j0 + i - 1;
+      p[i] = (j >= 0 && j < n) ? pos_of(a.v, q, j) : 0;
     }
-    if (c >= chunks_q) continue;
-    // members in earlier chunks
-    int32_t part = 0;
-    for (int i = threadIdx.x; i < c; i += blockDim.x) part += (int32_t)ccnt[i];
-    int32_t sum;
-    block_excl_scan(part, tmp, &sum);
-    if (threadIdx.x == 0) base_s = sum;
-    __syncthreads();
-    const int32_t base = base_s;
-    // this chunk: 16 consecutive candidates per thread, in index order
-    const int32_t j0 = c * kChunk + threadIdx.x * (kChunk / 256);
-    const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
-    uint32_t flags = 0;
+#pragma unroll
+    for (int i = 1; i <= kPer; ++i) {
+      const int32_t j = j0 + i - 1;
+      if (j > 0 && j < n && p[i] <= p[i - 1]) record_error(a.status, CSA2_ERR_ORDER);
+    }
+  }
+  for (int t = 0; t < a.n_k; ++t) {
+    const int32_t bstar = bst[t];
     int32_t cnt = 0;
 #pragma unroll
-    for (int i = 0; i < kChunk / 256; ++i) {
-      const int32_t j = j0 + i;
-      if (j < n && key_of(__ldg(sc + j), j) >= kth) {
-        flags |= 1u << i;
-        ++cnt;
+    for (int i = 0; i < kPer; ++i) cnt += bk[i] >= bstar && bk[i] > -2;
+    int32_t chunk_total;
+    const int32_t off = block_excl_scan(cnt, tmp, &chunk_total);
+    // publish this chunk's count, then add up the counts of the chunks before it
+    unsigned long long* pub =
+        reinterpret_cast<unsigned long long*>(a.s.chunk_cnt) + ((int64_t)q * 2 + t) * a.s.n_chunks;
+    if (threadIdx.x == 0) atomicExch(pub + c, (1ull << 32) | (uint32_t)chunk_total);
+    int32_t part = 0;
+    bool ok = true;
+    for (int i = threadIdx.x; i < c; i += blockDim.x) {
+      unsigned long long v = ld_relaxed_u64(pub + i);
+      if (!(v >> 32)) {
+        const uint64_t t0 = global_ns();
+        while (!((v = ld_relaxed_u64(pub + i)) >> 32)) {
+          if (global_ns() - t0 > kWaitLimitNs) {
+            ok = false;
+            break;
+          }
+        }
       }
+      part += (int32_t)(uint32_t)v;
     }
-    const int32_t off = block_excl_scan(cnt, tmp, nullptr);
-    int32_t w = base + off;
+    if (!ok) record_error(a.status, CSA2_ERR_TIMEOUT);
+    int32_t before;
+    block_excl_scan(part, tmp, &before);
+    if (threadIdx.x == 0) {
+      base_s = before;
+      const int32_t last = n > 0 ? (n - 1) / kChunk : 0;   // the chunk holding the last candidate
+      if (c == last) a.s.cand_cnt[q * 2 + t] = (uint32_t)(before + chunk_total);
+    }
+    __syncthreads();
+    int32_t w = base_s + off;
+    uint64_t* dst = a.s.cand + ((int64_t)q * 2 + t) * a.s.cand_cap;
 #pragma unroll
-    for (int i = 0; i < kChunk / 256; ++i) {
-      if (flags & (1u << i)) {
-        if (w < o.k) dst[w] = pos_of(a.v, q, j0 + i);
+    for (int i = 0; i < kPer; ++i) {
+      if (bk[i] >= bstar && bk[i] > -2) {
+        if (w < a.s.cand_cap) dst[w] = key_of(s[i], j0 + i);
         ++w;
       }
     }
     __syncthreads();
+  }
+}
+
+// ------------------------------------------------------------------ finish
+struct FinishArgs {
+  CandView v;
+  TopkScratch s;
+  TopkOut out[2];
+};
+
+constexpr int kTieCap = 2048;
+constexpr int kFinishPer = (kCandCap + 1023) / 1024;   // list keys per thread: i*1024 + thread
+
+// One CTA per (query, k).  The candidate list (position order) is loaded once
+// with all loads in flight, then every pass over it is a fully unrolled loop
+// over shared memory.  The ordered write uses per-(pass, warp) member counts,
+// as in the one-CTA kernel.
+__global__ void __launch_bounds__(1024, 1) topk_finish_kernel(FinishArgs a) {
+  extern __shared__ uint64_t keys_s[];            // [cand_cap] then [kTieCap] ties
+  uint64_t* ties = keys_s + kCandCap;
+  __shared__ int32_t cmat[kFinishPer * 32];
+  __shared__ uint32_t hist256[256];
+  __shared__ unsigned long long red[2];
+  __shared__ int32_t tmp[32];
+  __shared__ unsigned long long found;
+  const int q = blockIdx.x, t = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const TopkOut o = a.out[t];
+  const int32_t n = n_of(a.v, q);
+  const int32_t k = o.k;
+  const int32_t bstar = a.s.thresh[(q * 2 + t) * 2 + 0];
+  const int32_t above = a.s.thresh[(q * 2 + t) * 2 + 1];
+  const int32_t m = n > 0 ? (int32_t)a.s.cand_cnt[q * 2 + t] : 0;
+  int32_t* dst = o.idx + (int64_t)q * k;
+  const int32_t total = n < k ? n : k;
+  uint64_t kth = 0ull;
+  const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
+  if (m <= kCandCap) {
+    const unsigned long long* src =
+        reinterpret_cast<const unsigned long long*>(a.s.cand + ((int64_t)q * 2 + t) * a.s.cand_cap);
+    {
+      uint64_t r[kFinishPer];
+#pragma unroll
+      for (int i = 0; i < kFinishPer; ++i) {
+        const int32_t j = i * 1024 + tid;
+        r[i] = j < m ? __ldcg(src + j) : 0ull;
+      }
+#pragma unroll
+      for (int i = 0; i < kFinishPer; ++i) keys_s[i * 1024 + tid] = r[i];
+    }
+    __syncthreads();
+    if (bstar >= 0 && n > k) {
+      const int64_t need = (int64_t)k - above;
+      int32_t cnt = 0;
+#pragma unroll
+      for (int i = 0; i < kFinishPer; ++i) {
+        const int32_t j = i * 1024 + tid;
+        cnt += j < m && key_bucket(keys_s[j]) == bstar;
+      }
+      int32_t nt;
+      int32_t w = block_excl_scan(cnt, tmp, &nt);
+      if (nt <= kTieCap) {
+#pragma unroll
+        for (int i = 0; i < kFinishPer; ++i) {
+          const int32_t j = i * 1024 + tid;
+          if (j < m && key_bucket(keys_s[j]) == bstar) ties[w++] = keys_s[j];
+        }
+      }
+      if (tid == 0) found = 0ull;
+      __syncthreads();
+      if (nt <= 1024) {   // exact rank among the ties
+        if (tid < nt) {
+          const uint64_t ki = ties[tid];
+          int32_t above_i = 0;
+          for (int32_t j = 0; j < nt; ++j) above_i += ties[j] > ki;
+          if (above_i == need - 1) found = ki;
+        }
+        __syncthreads();
+        kth = found;
+      } else if (nt <= kTieCap) {
+        kth = radix_select([&](int64_t i) { return ties[i]; }, nt, need, hist256, red);
+      } else {
+        kth = radix_select([&](int64_t i) { return key_bucket(keys_s[i]) == bstar ? keys_s[i] : 0ull; }, m,
+                           need, hist256, red);
+      }
+    }
+    uint32_t mem = 0;
+#pragma unroll
+    for (int i = 0; i < kFinishPer; ++i) {
+      const int32_t j = i * 1024 + tid;
+      const bool in = j < m && keys_s[j] >= kth;
+      mem |= (uint32_t)in << i;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (lane == 0) cmat[i * 32 + warp] = __popc(bal);
+    }
+    __syncthreads();
+    const int32_t cval = tid < kFinishPer * 32 ? cmat[tid] : 0;
+    const int32_t cbase = block_excl_scan(cval, tmp, nullptr);
+    if (tid < kFinishPer * 32) cmat[tid] = cbase;
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kFinishPer; ++i) {
+      const int32_t j = i * 1024 + tid;
+      const bool in = (mem >> i) & 1u;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      const int32_t slot = cmat[i * 32 + warp] + __popc(bal & ((1u << lane) - 1u));
+      if (in && slot < k) dst[slot] = pos_of(a.v, q, key_index(keys_s[j]));
+    }
+  } else {
+    // The list overflowed (a very flat score distribution): select and compact
+    // over the whole score row instead.
+    auto get = [&](int64_t j) -> uint64_t {
+      const int32_t s = __ldg(sc + j);
+      return (int32_t)score_bucket(s) == bstar ? key_of(s, (int32_t)j) : 0ull;
+    };
+    if (bstar >= 0 && n > k) kth = radix_select(get, n, (int64_t)k - above, hist256, red);
+    __shared__ int32_t run;
+    if (tid == 0) run = 0;
+    __syncthreads();
+    for (int32_t base = 0; base < n; base += 1024 * 8) {
+      const int32_t j0 = base + tid * 8;
+      int32_t cnt = 0;
+      for (int i = 0; i < 8; ++i) cnt += (j0 + i < n) && key_of(__ldg(sc + j0 + i), j0 + i) >= kth;
+      int32_t tot;
+      int32_t w = run + block_excl_scan(cnt, tmp, &tot);
+      for (int i = 0; i < 8; ++i) {
+        const int32_t j = j0 + i;
+        if (j < n && key_of(__ldg(sc + j), j) >= kth) {
+          if (w < k) dst[w] = pos_of(a.v, q, j);
+          ++w;
+        }
+      }
+      __syncthreads();
+      if (tid == 0) run += tot;
+      __syncthreads();
+    }
+  }
+  for (int32_t i = total + tid; i < k; i += 1024) dst[i] = -1;
+  if (tid == 0) {
+    if (o.cnt) o.cnt[q] = total;
+    a.s.kth[q * 2 + t] = kth;
   }
 }
 
@@ -438,43 +559,118 @@ struct SmallArgs {
   int32_t* status;
 };
 
-__global__ void __launch_bounds__(1024) topk_small_kernel(SmallArgs a) {
-  extern __shared__ uint64_t keys_s[];   // [n]
+constexpr int kSmallTieCap = 2048;
+constexpr int kSmallPer = kSmallMax / 1024;   // candidates per thread: j = i*1024 + thread
+
+// One CTA per query, up to kSmallMax candidates.  Each thread keeps its
+// scores (and candidate positions) in registers from the first, fully
+// overlapped load round on.  Shared memory holds only the histogram, the
+// ties and a count per (pass, warp) for the ordered write.
+__global__ void __launch_bounds__(1024, 1) topk_small_kernel(SmallArgs a) {
+  extern __shared__ uint64_t small_dyn[];                                   // ties, then the histogram
+  uint64_t* ties = small_dyn;                                              // [kSmallTieCap]
+  uint32_t* hist = reinterpret_cast<uint32_t*>(small_dyn + kSmallTieCap);  // [kBuckets]
+  __shared__ int32_t cmat[kSmallPer * 32];
   __shared__ uint32_t hist256[256];
   __shared__ unsigned long long red[2];
   __shared__ int32_t tmp[32];
-  const int q = blockIdx.x;
+  __shared__ int32_t bstar_s, above_s;
+  __shared__ unsigned long long found;
+  const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int32_t n = n_of(a.v, q);
   const int32_t k = a.k;
   int32_t* dst = a.out_idx + (int64_t)q * k;
   const int32_t total = n < k ? n : k;
   const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
-  for (int32_t j = threadIdx.x; j < n; j += blockDim.x) {
-    keys_s[j] = key_of(__ldg(sc + j), j);
-    if (a.v.cand_pos && j > 0 && pos_of(a.v, q, j) <= pos_of(a.v, q, j - 1))
-      record_error(a.status, CSA2_ERR_ORDER);
+  const int32_t* cp = a.v.cand_pos ? a.v.cand_pos + (int64_t)q * a.v.ld : nullptr;
+  int32_t sr[kSmallPer], pr[kSmallPer];
+#pragma unroll
+  for (int i = 0; i < kSmallPer; ++i) {
+    const int32_t j = i * 1024 + tid;
+    sr[i] = j < n ? __ldg(sc + j) : 0;
+    pr[i] = cp ? (j < n ? __ldg(cp + j) : 0) : j;
+  }
+  for (int i = tid; i < kBuckets; i += 1024) hist[i] = 0;
+  if (cp) {   // candidate positions must ascend (lane 0 reads its left neighbour itself)
+#pragma unroll
+    for (int i = 0; i < kSmallPer; ++i) {
+      const int32_t j = i * 1024 + tid;
+      int32_t pp = __shfl_up_sync(0xffffffffu, pr[i], 1);
+      if (lane == 0) pp = (j > 0 && j < n) ? __ldg(cp + j - 1) : -1;
+      if (j > 0 && j < n && pr[i] <= pp) record_error(a.status, CSA2_ERR_ORDER);
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kSmallPer; ++i) {
+    const int32_t j = i * 1024 + tid;
+    if (j < n) atomicAdd(&hist[score_bucket(sr[i])], 1u);   // buckets spread: plain atomics beat aggregation
   }
   __syncthreads();
   uint64_t kth = 0ull;
-  if (n > k) kth = radix_select([&](int64_t i) { return keys_s[i]; }, n, k, hist256, red);
-  // stable compaction: ceil(n / 1024) consecutive candidates per thread
-  const int32_t per = (n + blockDim.x - 1) / blockDim.x;
-  const int32_t j0 = threadIdx.x * per;
-  int32_t cnt = 0;
-  for (int32_t i = 0; i < per; ++i) {
-    const int32_t j = j0 + i;
-    if (j < n && keys_s[j] >= kth) ++cnt;
-  }
-  int32_t w = block_excl_scan(cnt, tmp, nullptr);
-  for (int32_t i = 0; i < per; ++i) {
-    const int32_t j = j0 + i;
-    if (j < n && keys_s[j] >= kth) {
-      if (w < k) dst[w] = pos_of(a.v, q, j);
-      ++w;
+  if (n > k) {
+    find_threshold<1024>(hist, k, &bstar_s, &above_s, tmp);
+    const int32_t bstar = bstar_s;
+    const int64_t need = (int64_t)k - above_s;
+    int32_t cnt = 0;
+#pragma unroll
+    for (int i = 0; i < kSmallPer; ++i) cnt += (i * 1024 + tid < n) && (int32_t)score_bucket(sr[i]) == bstar;
+    int32_t nt;
+    int32_t w = block_excl_scan(cnt, tmp, &nt);
+    if (nt <= kSmallTieCap) {
+#pragma unroll
+      for (int i = 0; i < kSmallPer; ++i) {
+        const int32_t j = i * 1024 + tid;
+        if (j < n && (int32_t)score_bucket(sr[i]) == bstar) ties[w++] = key_of(sr[i], j);
+      }
+    }
+    if (tid == 0) found = 0ull;
+    __syncthreads();
+    if (nt <= 1024) {   // exact rank among the ties
+      if (tid < nt) {
+        const uint64_t ki = ties[tid];
+        int32_t above = 0;
+        for (int32_t j = 0; j < nt; ++j) above += ties[j] > ki;
+        if (above == need - 1) found = ki;
+      }
+      __syncthreads();
+      kth = found;
+    } else if (nt <= kSmallTieCap) {
+      kth = radix_select([&](int64_t i) { return ties[i]; }, nt, need, hist256, red);
+    } else {
+      kth = radix_select(
+          [&](int64_t j) -> uint64_t {
+            const int32_t s = __ldg(sc + j);
+            return (int32_t)score_bucket(s) == bstar ? key_of(s, (int32_t)j) : 0ull;
+          },
+          n, need, hist256, red);
     }
   }
-  for (int32_t i = total + threadIdx.x; i < k; i += blockDim.x) dst[i] = -1;
-  if (threadIdx.x == 0 && a.out_cnt) a.out_cnt[q] = total;
+  // ordered write: candidate j = i*1024 + warp*32 + lane, so (i, warp, lane)
+  // is position order; count members per (i, warp), scan, then place
+  uint32_t mem = 0;   // bit i: candidate i*1024 + tid is a member
+#pragma unroll
+  for (int i = 0; i < kSmallPer; ++i) {
+    const int32_t j = i * 1024 + tid;
+    const bool in = j < n && key_of(sr[i], j) >= kth;
+    mem |= (uint32_t)in << i;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    if (lane == 0) cmat[i * 32 + warp] = __popc(bal);
+  }
+  __syncthreads();
+  const int32_t cval = tid < kSmallPer * 32 ? cmat[tid] : 0;
+  const int32_t cbase = block_excl_scan(cval, tmp, nullptr);
+  if (tid < kSmallPer * 32) cmat[tid] = cbase;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kSmallPer; ++i) {
+    const bool in = (mem >> i) & 1u;
+    const uint32_t bal = __ballot_sync(0xffffffffu, in);
+    const int32_t slot = cmat[i * 32 + warp] + __popc(bal & ((1u << lane) - 1u));
+    if (in && slot < k) dst[slot] = pr[i];
+  }
+  for (int32_t i = total + tid; i < k; i += 1024) dst[i] = -1;
+  if (tid == 0 && a.out_cnt) a.out_cnt[q] = total;
 }
 
 }  // namespace
@@ -492,17 +688,18 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
     if (e != cudaSuccess) return e;
     topk_hist_kernel<<<grid, 256, 0, st>>>(v, s.hist);
   }
-  e = cudaMemsetAsync(s.cand_cnt, 0, (size_t)nq * 2 * sizeof(uint32_t), st);
+  e = cudaMemsetAsync(s.chunk_cnt, 0, (size_t)nq * 2 * s.n_chunks * 8, st);
   if (e != cudaSuccess) return e;
-  SelectArgs sa{v, s, {outs[0].k, n_k > 1 ? outs[1].k : 0}, n_k, status};
-  topk_select_kernel<<<grid, 256, 0, st>>>(sa);
+  ThreshArgs ta{s, {outs[0].k, n_k > 1 ? outs[1].k : 0}, n_k};
+  topk_thresh_kernel<<<nq, 256, 0, st>>>(ta);
+  GatherArgs ga{v, s, n_k, status};
+  topk_gather_kernel<<<grid, 256, 0, st>>>(ga);
+  const int smem = (kCandCap + kTieCap) * 8;
   static unsigned long long done = 0;
-  e = ensure_smem(topk_resolve_kernel, kResolveSmemKeys * 8, done);
+  e = ensure_smem(topk_finish_kernel, smem, done);
   if (e != cudaSuccess) return e;
-  ResolveArgs ra{v, s, {outs[0].k, n_k > 1 ? outs[1].k : 0}};
-  topk_resolve_kernel<<<dim3(nq, n_k), 1024, kResolveSmemKeys * 8, st>>>(ra);
-  WriteArgs wa{v, s, {outs[0], n_k > 1 ? outs[1] : outs[0]}, n_k};
-  topk_write_kernel<<<grid, 256, 0, st>>>(wa);
+  FinishArgs fa{v, s, {outs[0], n_k > 1 ? outs[1] : outs[0]}};
+  topk_finish_kernel<<<dim3(nq, n_k), 1024, smem, st>>>(fa);
   return cudaGetLastError();
 }
 
@@ -510,12 +707,12 @@ cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* 
                               const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                               int32_t* out_idx, int32_t* out_cnt, int32_t* status,
                               cudaStream_t st) {
+  const int smem = kSmallTieCap * 8 + kBuckets * 4;
   static unsigned long long done = 0;
-  cudaError_t e = ensure_smem(topk_small_kernel, kSmallMax * 8, done);
+  cudaError_t e = ensure_smem(topk_small_kernel, smem, done);
   if (e != cudaSuccess) return e;
   CandView v{scores, ld, n_valid, nullptr, cand_pos, n_max};
   SmallArgs sa{v, k, out_idx, out_cnt, status};
-  const size_t smem = (size_t)(n_max > 0 ? n_max : 1) * 8;
   topk_small_kernel<<<nq, 1024, smem, st>>>(sa);
   return cudaGetLastError();
 }

@@ -294,3 +294,23 @@ def test_plan_repeat_is_deterministic():
     torch.cuda.synchronize()
     for a, ly in zip(first, c.layers_dev):
         assert torch.equal(a, ly.out)
+
+
+def test_sparse_attention_long_selection():
+    # K = 2000 > the 1024 selection entries a CTA keeps in shared memory,
+    # and more than 24 chunks of 64 rows for the combine.
+    wl = synth.scaled(synth.C0_TINY, seq_lens=(6000,), topk=2000, pool=3000)
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    pos = int(c.query_pos[0])
+    q, w = c.host_q[(0, 0)]
+    _, _, sel = O.full_index(q, w, c.host_keys[(0, 0)], pos, wl.pool, wl.topk)
+    sel_d = torch.from_numpy(sel.astype(np.int32)[None]).to(DEV)
+    B.check_status(B.csa2_sparse_attn_fp4(ly.q_attn, ly.codes, ly.scales, c.pos_dev, sel_d, ly.out,
+                                          sel_cnt=torch.tensor([len(sel)], dtype=torch.int32, device=DEV),
+                                          window=wl.window))
+    S = O.attention_set(sel, pos, wl.window)
+    codes, scales = c.fp4_host[(0, 0)]
+    ref, _ = O.sparse_attention(c.host_qa[(0, 0)], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
+    ok, err = G.tol_ok(_np(ly.out.float())[0], ref)
+    assert ok, f"max abs err {err}"

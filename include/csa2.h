@@ -163,7 +163,7 @@ size_t csa2_topk_pool_workspace(int32_t nq, int32_t n_max, int32_t k);
  * n_max <= 16384 needs no scratch.  Larger sizes must satisfy
  * csa2_topk_pool_workspace(nq, n_max, k) <= CSA2_NOALLOC_SCRATCH_BYTES;
  * otherwise the call returns CSA2_ERR_WORKSPACE and launches nothing.  That
- * allows 9 queries of up to 10^6 candidates each, or 8 of up to 2^24.
+ * allows 8 queries of up to 10^6 candidates each, or 7 of up to 2^24.
  * The call allocates and frees nothing.  Its first call on a device looks up
  * the array's address there (cudaGetSymbolAddress), so make that first call
  * before any stream capture on that device.

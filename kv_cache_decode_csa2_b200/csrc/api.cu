@@ -97,7 +97,7 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   const int64_t ld = scores ? ld_scores : max_ctx;
   const bool topk = P > 0 || K > 0;
   if (topk) {
-    cudaError_t e = cudaMemsetAsync(ts.hist, 0, (size_t)nq * kBuckets * sizeof(uint32_t), st);
+    cudaError_t e = cudaMemsetAsync(ts.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
   }
   cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,

@@ -31,11 +31,27 @@ struct TopkScratch {
   uint32_t* cand_cnt;    // [nq][2]
   uint64_t* kth;         // [nq][2]                        key of the k-th best candidate
   int32_t* thresh;       // [nq][2][2]                     bucket b*, members above b*
+  uint32_t* sel_hdr;     // [nq][4]    select: barrier count, tie counts (follows hist; zeroed with it)
+  uint64_t* sel_ties;    // [nq][2][kSelTieCap]            select: ties of the threshold bucket
+  uint32_t* sel_mcnt;    // [nq][2][kSelMaxG]              select: members per CTA
+  uint32_t* sel_radix;   // [nq][2][8][256]                select: digit counts (flat distributions)
   int32_t n_chunks;
   int32_t cand_cap;
 };
 constexpr int kChunk = 4096;          // positions per chunk in the multi-CTA passes
 constexpr int kCandCap = 24576;       // ordered candidates (bucket >= b*) kept per (query, k)
+
+// Select kernel (topk_select.cu): one CTA of kSelNT threads per kSelSpan
+// candidates of a row; rows of more than kSelSpan candidates use co-resident
+// CTAs that meet at grid barriers.
+constexpr int kSelNT = 1024;
+constexpr int kSelPer = 16;
+constexpr int kSelSpan = kSelNT * kSelPer;
+constexpr int kSelTieCap = 4096;
+constexpr int kSelMaxG = 256;
+// Bytes from TopkScratch::hist that must be zero before the histogram pass
+// and the select kernel (the histograms and the select header).
+inline size_t topk_zero_bytes(int32_t nq) { return (size_t)nq * (kBuckets + 4) * sizeof(uint32_t); }
 
 size_t topk_scratch_bytes(int32_t nq, int32_t n_max);
 TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);
@@ -62,12 +78,24 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
                               const TopkScratch& s, bool hist_ready, int32_t* status,
                               cudaStream_t st);
 
-// Single-CTA-per-query top-k for up to kSmallMax candidates.
+// Top-k for up to kSmallMax candidates per query: one select CTA per query.
 constexpr int kSmallMax = 16384;
+static_assert(kSmallMax <= kSelSpan, "the small path is one select CTA per query");
 cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* n_valid,
                               const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                               int32_t* out_idx, int32_t* out_cnt, int32_t* status,
                               cudaStream_t st);
+
+// Exact top-k of nq score rows in position order, for one or two k.  hist,
+// when given, is the complete bucket histogram of each row and s the scratch
+// whose select header is zero; without them n_max must be at most kSelSpan.
+// Returns cudaErrorNotSupported when the rows need more CTAs than fit on the
+// device at once (the caller then takes the multi-pass path).
+cudaError_t launch_select(const int32_t* scores, int64_t ld, const int32_t* n_valid,
+                          const int32_t* query_pos, const int32_t* cand_pos, int32_t nq, int32_t n_max,
+                          const TopkOut* outs, int32_t n_k, const uint32_t* hist, const TopkScratch* s,
+                          int32_t* status, cudaStream_t st);
+
 
 // K3 scoring part: scores of the pool entries (slot order) for each query.
 cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,

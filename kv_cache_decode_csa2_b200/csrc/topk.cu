@@ -15,16 +15,21 @@
 // ties finds it, and a stable compaction writes the members in position
 // order.  No sort is needed.
 //
-// Large n (multi-CTA):
+// Passes:
 //   hist    bucket histogram (fused into the index-score kernel when the scores
 //           come from there)
-//   gather  one CTA per 4096-candidate chunk: finds b* from the histogram,
-//           counts the chunk's candidates with bucket >= b*, publishes the
-//           count, adds up the counts of the chunks before it (bounded wait),
-//           and writes those candidates' keys in position order
+//   select  (topk_select.cu) when the rows fit on the device at once: the
+//           whole selection in one launch of co-resident CTAs; it is also the
+//           small-n path (n <= kSmallMax, one CTA per query)
+// Otherwise, the multi-pass path:
+//   thresh  one CTA per query finds b* from the histogram
+//   gather  one CTA per 4096-candidate chunk counts the chunk's candidates
+//           with bucket >= b*, publishes the count, adds up the counts of the
+//           chunks before it (bounded wait), and writes those candidates' keys
+//           in position order
 //   finish  one CTA per (query, k): radix select of the k-th key among the
 //           ties of its ordered candidate list, then the ordered compaction
-// Small n (<= kSmallMax): one CTA per query does all of this in shared memory.
+//           (a list that overflowed its capacity is redone from the score row)
 // Bucket histograms use plain shared atomics (scores spread over many buckets);
 // the digit histograms of the radix select, where lanes collide, are warp-aggregated.
 #include "csa2_device.cuh"
@@ -44,11 +49,15 @@ TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max) {
   if (s.n_chunks < 1) s.n_chunks = 1;
   s.cand_cap = kCandCap;
   s.hist = c.take<uint32_t>((size_t)nq * kBuckets);
+  s.sel_hdr = c.take<uint32_t>((size_t)nq * 4);   // directly after hist: one memset zeroes both
   s.chunk_cnt = c.take<uint32_t>((size_t)nq * 2 * s.n_chunks * 2);   // published (flag, count) pairs
   s.cand = c.take<uint64_t>((size_t)nq * 2 * s.cand_cap);
   s.cand_cnt = c.take<uint32_t>((size_t)nq * 2);
   s.kth = c.take<uint64_t>((size_t)nq * 2);
   s.thresh = c.take<int32_t>((size_t)nq * 4);
+  s.sel_ties = c.take<uint64_t>((size_t)nq * 2 * kSelTieCap);
+  s.sel_mcnt = c.take<uint32_t>((size_t)nq * 2 * kSelMaxG);
+  s.sel_radix = c.take<uint32_t>((size_t)nq * 2 * 8 * 256);
   return s;
 }
 
@@ -550,129 +559,6 @@ __global__ void __launch_bounds__(1024, 1) topk_finish_kernel(FinishArgs a) {
   }
 }
 
-// ------------------------------------------------------------------ small: one CTA per query
-struct SmallArgs {
-  CandView v;
-  int32_t k;
-  int32_t* out_idx;
-  int32_t* out_cnt;
-  int32_t* status;
-};
-
-constexpr int kSmallTieCap = 2048;
-constexpr int kSmallPer = kSmallMax / 1024;   // candidates per thread: j = i*1024 + thread
-
-// One CTA per query, up to kSmallMax candidates.  Each thread keeps its
-// scores (and candidate positions) in registers from the first, fully
-// overlapped load round on.  Shared memory holds only the histogram, the
-// ties and a count per (pass, warp) for the ordered write.
-__global__ void __launch_bounds__(1024, 1) topk_small_kernel(SmallArgs a) {
-  extern __shared__ uint64_t small_dyn[];                                   // ties, then the histogram
-  uint64_t* ties = small_dyn;                                              // [kSmallTieCap]
-  uint32_t* hist = reinterpret_cast<uint32_t*>(small_dyn + kSmallTieCap);  // [kBuckets]
-  __shared__ int32_t cmat[kSmallPer * 32];
-  __shared__ uint32_t hist256[256];
-  __shared__ unsigned long long red[2];
-  __shared__ int32_t tmp[32];
-  __shared__ int32_t bstar_s, above_s;
-  __shared__ unsigned long long found;
-  const int q = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int32_t n = n_of(a.v, q);
-  const int32_t k = a.k;
-  int32_t* dst = a.out_idx + (int64_t)q * k;
-  const int32_t total = n < k ? n : k;
-  const int32_t* sc = a.v.scores + (int64_t)q * a.v.ld;
-  const int32_t* cp = a.v.cand_pos ? a.v.cand_pos + (int64_t)q * a.v.ld : nullptr;
-  int32_t sr[kSmallPer], pr[kSmallPer];
-#pragma unroll
-  for (int i = 0; i < kSmallPer; ++i) {
-    const int32_t j = i * 1024 + tid;
-    sr[i] = j < n ? __ldg(sc + j) : 0;
-    pr[i] = cp ? (j < n ? __ldg(cp + j) : 0) : j;
-  }
-  for (int i = tid; i < kBuckets; i += 1024) hist[i] = 0;
-  if (cp) {   // candidate positions must ascend (lane 0 reads its left neighbour itself)
-#pragma unroll
-    for (int i = 0; i < kSmallPer; ++i) {
-      const int32_t j = i * 1024 + tid;
-      int32_t pp = __shfl_up_sync(0xffffffffu, pr[i], 1);
-      if (lane == 0) pp = (j > 0 && j < n) ? __ldg(cp + j - 1) : -1;
-      if (j > 0 && j < n && pr[i] <= pp) record_error(a.status, CSA2_ERR_ORDER);
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < kSmallPer; ++i) {
-    const int32_t j = i * 1024 + tid;
-    if (j < n) atomicAdd(&hist[score_bucket(sr[i])], 1u);   // buckets spread: plain atomics beat aggregation
-  }
-  __syncthreads();
-  uint64_t kth = 0ull;
-  if (n > k) {
-    find_threshold<1024>(hist, k, &bstar_s, &above_s, tmp);
-    const int32_t bstar = bstar_s;
-    const int64_t need = (int64_t)k - above_s;
-    int32_t cnt = 0;
-#pragma unroll
-    for (int i = 0; i < kSmallPer; ++i) cnt += (i * 1024 + tid < n) && (int32_t)score_bucket(sr[i]) == bstar;
-    int32_t nt;
-    int32_t w = block_excl_scan(cnt, tmp, &nt);
-    if (nt <= kSmallTieCap) {
-#pragma unroll
-      for (int i = 0; i < kSmallPer; ++i) {
-        const int32_t j = i * 1024 + tid;
-        if (j < n && (int32_t)score_bucket(sr[i]) == bstar) ties[w++] = key_of(sr[i], j);
-      }
-    }
-    if (tid == 0) found = 0ull;
-    __syncthreads();
-    if (nt <= 1024) {   // exact rank among the ties
-      if (tid < nt) {
-        const uint64_t ki = ties[tid];
-        int32_t above = 0;
-        for (int32_t j = 0; j < nt; ++j) above += ties[j] > ki;
-        if (above == need - 1) found = ki;
-      }
-      __syncthreads();
-      kth = found;
-    } else if (nt <= kSmallTieCap) {
-      kth = radix_select([&](int64_t i) { return ties[i]; }, nt, need, hist256, red);
-    } else {
-      kth = radix_select(
-          [&](int64_t j) -> uint64_t {
-            const int32_t s = __ldg(sc + j);
-            return (int32_t)score_bucket(s) == bstar ? key_of(s, (int32_t)j) : 0ull;
-          },
-          n, need, hist256, red);
-    }
-  }
-  // ordered write: candidate j = i*1024 + warp*32 + lane, so (i, warp, lane)
-  // is position order; count members per (i, warp), scan, then place
-  uint32_t mem = 0;   // bit i: candidate i*1024 + tid is a member
-#pragma unroll
-  for (int i = 0; i < kSmallPer; ++i) {
-    const int32_t j = i * 1024 + tid;
-    const bool in = j < n && key_of(sr[i], j) >= kth;
-    mem |= (uint32_t)in << i;
-    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-    if (lane == 0) cmat[i * 32 + warp] = __popc(bal);
-  }
-  __syncthreads();
-  const int32_t cval = tid < kSmallPer * 32 ? cmat[tid] : 0;
-  const int32_t cbase = block_excl_scan(cval, tmp, nullptr);
-  if (tid < kSmallPer * 32) cmat[tid] = cbase;
-  __syncthreads();
-#pragma unroll
-  for (int i = 0; i < kSmallPer; ++i) {
-    const bool in = (mem >> i) & 1u;
-    const uint32_t bal = __ballot_sync(0xffffffffu, in);
-    const int32_t slot = cmat[i * 32 + warp] + __popc(bal & ((1u << lane) - 1u));
-    if (in && slot < k) dst[slot] = pr[i];
-  }
-  for (int32_t i = total + tid; i < k; i += 1024) dst[i] = -1;
-  if (tid == 0 && a.out_cnt) a.out_cnt[q] = total;
-}
-
 }  // namespace
 
 cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* n_valid,
@@ -684,10 +570,14 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
   const dim3 grid(s.n_chunks, nq);
   cudaError_t e;
   if (!hist_ready) {
-    e = cudaMemsetAsync(s.hist, 0, (size_t)nq * kBuckets * sizeof(uint32_t), st);
+    e = cudaMemsetAsync(s.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return e;
     topk_hist_kernel<<<grid, 256, 0, st>>>(v, s.hist);
   }
+  // One pass of co-resident select CTAs when the rows fit on the device.
+  e = launch_select(scores, ld, n_valid, query_pos, cand_pos, nq, n_max, outs, n_k, s.hist, &s, status, st);
+  if (e != cudaErrorNotSupported) return e;
+  (void)cudaGetLastError();
   e = cudaMemsetAsync(s.chunk_cnt, 0, (size_t)nq * 2 * s.n_chunks * 8, st);
   if (e != cudaSuccess) return e;
   ThreshArgs ta{s, {outs[0].k, n_k > 1 ? outs[1].k : 0}, n_k};
@@ -707,14 +597,8 @@ cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* 
                               const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                               int32_t* out_idx, int32_t* out_cnt, int32_t* status,
                               cudaStream_t st) {
-  const int smem = kSmallTieCap * 8 + kBuckets * 4;
-  static unsigned long long done = 0;
-  cudaError_t e = ensure_smem(topk_small_kernel, smem, done);
-  if (e != cudaSuccess) return e;
-  CandView v{scores, ld, n_valid, nullptr, cand_pos, n_max};
-  SmallArgs sa{v, k, out_idx, out_cnt, status};
-  topk_small_kernel<<<nq, 1024, smem, st>>>(sa);
-  return cudaGetLastError();
+  const TopkOut o{out_idx, out_cnt, k};
+  return launch_select(scores, ld, n_valid, nullptr, cand_pos, nq, n_max, &o, 1, nullptr, nullptr, status, st);
 }
 
 }  // namespace csa2

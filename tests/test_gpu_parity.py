@@ -135,8 +135,12 @@ def test_index_bad_position_is_reported():
 
 
 # ------------------------------------------------------------------ K2: top-k alone
+# Sizes cover one select CTA per row (n <= 16384), several co-resident CTAs per
+# row (n > 16384), and rows that do not fit on the device at once (3 x 10^6:
+# the multi-pass path); spreads 2 and 3 make tie lists too long to rank.
 @pytest.mark.parametrize("n,k,spread", [(5000, 700, 3), (16384, 512, 50), (16385, 512, 50),
-                                        (70000, 16384, 1000), (70000, 300, 2), (300000, 16384, 10 ** 6)])
+                                        (70000, 16384, 1000), (70000, 300, 2), (300000, 16384, 10 ** 6),
+                                        (1000000, 16384, 25000)])
 def test_topk_pool_matches_oracle(n, k, spread):
     rng = np.random.default_rng(n + k)
     nq = 3
@@ -153,7 +157,7 @@ def test_topk_pool_matches_oracle(n, k, spread):
         assert (o[i, c[i]:] == -1).all()
 
 
-@pytest.mark.parametrize("n", [1000, 40000])
+@pytest.mark.parametrize("n", [1000, 16000, 40000])
 def test_topk_all_equal_and_two_valued(n):
     for s in (np.zeros((1, n), np.int32), np.where(np.arange(n) % 3 == 0, 7, -7).astype(np.int32)[None]):
         k = 600

@@ -38,14 +38,50 @@ size_t index_full_ws(int32_t nq, int32_t max_ctx, int32_t P, int32_t K, void* ba
   return c.used + 256;
 }
 
-size_t reindex_ws(int32_t nq, int32_t P, void* base, int32_t** scores, TopkScratch* ts) {
+// Reindex scratch for n_jobs layers over one pool: the fused launch's
+// histograms and lists, and (for batches too large to be co-resident) one
+// layer's scores and top-k scratch, reused layer after layer.
+size_t reindex_ws(int32_t nq, int32_t P, int32_t n_jobs, void* base, int32_t** scores, TopkScratch* ts,
+                  ReindexSelScratch* rs) {
   Carver c(base);
+  ReindexSelScratch r = carve_reindex_select(c, nq * n_jobs, P);
   int32_t* sc = c.take<int32_t>((size_t)nq * (size_t)P);
   TopkScratch t{};
   if (P > kSmallMax) t = carve_topk(c, nq, P);
   if (scores) *scores = sc;
   if (ts) *ts = t;
+  if (rs) *rs = r;
   return c.used + 256;
+}
+
+// Scores and top-K of reindex layers that search the same pool: one fused
+// launch when its CTAs fit on the device at once, else per layer a scoring
+// launch and a select launch.
+int32_t run_reindex(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* seq_of_query,
+                    const int32_t* pool_idx, const int32_t* pool_cnt, int32_t nq, int32_t H, int32_t D, int32_t P,
+                    int32_t K, void* ws, int32_t* status, cudaStream_t st) {
+  int32_t* sc_ws;
+  TopkScratch ts;
+  ReindexSelScratch rs;
+  reindex_ws(nq, P, n_jobs, ws, &sc_ws, &ts, &rs);
+  cudaError_t e = launch_reindex_select(jobs, n_jobs, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, K, rs,
+                                        status, st);
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+  (void)cudaGetLastError();
+  for (int j = 0; j < n_jobs; ++j) {
+    const ReindexJobDesc& d = jobs[j];
+    int32_t* sc = d.scores ? d.scores : sc_ws;
+    e = launch_reindex_score(d.q, d.w, *d.keys, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, sc, status, st);
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+    if (P <= kSmallMax) {
+      e = launch_topk_small(sc, P, pool_cnt, pool_idx, nq, P, K, d.sel_idx, d.sel_cnt, status, st);
+    } else {
+      TopkOut o{d.sel_idx, d.sel_cnt, K};
+      e = launch_topk_large(sc, P, pool_cnt, nullptr, pool_idx, nq, P, &o, 1, ts, false, status, st);
+    }
+    if (e != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  return CSA2_OK;
 }
 
 }  // namespace
@@ -142,7 +178,7 @@ int32_t csa2_topk_pool(const int32_t* scores, int64_t ld, const int32_t* n_valid
 size_t csa2_reindex_workspace(int32_t nq, int32_t P, int32_t K) {
   (void)K;
   if (nq < 1 || P < 1) return 0;
-  return reindex_ws(nq, P, nullptr, nullptr, nullptr);
+  return reindex_ws(nq, P, 1, nullptr, nullptr, nullptr, nullptr);
 }
 
 int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
@@ -157,19 +193,9 @@ int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   if (H < 1 || H > 128) return CSA2_ERR_UNSUPPORTED;
   if (!rows_ok(keys, D, 16)) return CSA2_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < csa2_reindex_workspace(nq, P, K)) return CSA2_ERR_WORKSPACE;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int32_t* sc_ws;
-  TopkScratch ts;
-  reindex_ws(nq, P, ws, &sc_ws, &ts);
-  int32_t* sc = scores ? scores : sc_ws;
-  cudaError_t e = launch_reindex_score(q, w, *keys, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, sc,
-                                       status, st);
-  if (e != cudaSuccess) return CSA2_ERR_CUDA;
-  if (P <= kSmallMax)
-    return cuda_status(launch_topk_small(sc, P, pool_cnt, pool_idx, nq, P, K, sel_idx, sel_cnt, status, st));
-  TopkOut o{sel_idx, sel_cnt, K};
-  return cuda_status(launch_topk_large(sc, P, pool_cnt, nullptr, pool_idx, nq, P, &o, 1, ts, false,
-                                       status, st));
+  const ReindexJobDesc job{q, w, keys, scores, sel_idx, sel_cnt};
+  return run_reindex(&job, 1, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, K, ws, status,
+                     static_cast<cudaStream_t>(stream));
 }
 
 size_t csa2_sparse_attn_workspace(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window) {
@@ -224,9 +250,10 @@ PlanWs carve_plan(const int32_t* modes, int32_t L, const csa2_plan_shape* s, voi
   Carver c(base);
   p.index_ws = csa2_index_full_workspace(s->nq, s->max_ctx, s->P, s->K);
   p.index_base = c.take<char>(p.index_ws);
-  bool any_reindex = false;
-  for (int i = 0; i < L; ++i) any_reindex |= modes[i] == CSA2_REINDEX;
-  p.reindex_ws = any_reindex ? csa2_reindex_workspace(s->nq, s->P, s->K) : 0;
+  int n_reindex = 0;
+  for (int i = 0; i < L; ++i) n_reindex += modes[i] == CSA2_REINDEX;
+  const int group = n_reindex < kMaxReindexJobs ? n_reindex : kMaxReindexJobs;
+  p.reindex_ws = group ? reindex_ws(s->nq, s->P, group, nullptr, nullptr, nullptr, nullptr) : 0;
   p.reindex_base = c.take<char>(p.reindex_ws);
   p.attn_ws = csa2_sparse_attn_workspace(s->nq, s->Hq, s->D, s->K, s->window) * (size_t)L;
   p.attn_base = c.take<char>(p.attn_ws);
@@ -282,43 +309,70 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
   PlanWs p = carve_plan(modes, L, s, ws);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  AttnJobDesc jobs[kMaxAttnJobs];
-  int32_t* cur_pool = nullptr;
-  int32_t* cur_pool_cnt = nullptr;
-  int32_t* cur_sel = nullptr;
-  int32_t* cur_sel_cnt = nullptr;
+  // Which buffers every layer reads and writes.  A REINDEX layer searches the
+  // pool of the latest FULL layer; a REUSE layer attends to the selection of
+  // the latest FULL or REINDEX layer.
+  int32_t* pool_of[kMaxAttnJobs];
+  int32_t* pool_cnt_of[kMaxAttnJobs];
+  int32_t* sel_of[kMaxAttnJobs];
+  int32_t* sel_cnt_of[kMaxAttnJobs];
   for (int i = 0; i < L; ++i) {
     const csa2_layer& ly = layers[i];
     if (modes[i] == CSA2_FULL) {
-      cur_pool = ly.pool_idx ? ly.pool_idx : p.pool[i];
-      cur_pool_cnt = ly.pool_cnt ? ly.pool_cnt : p.pool_cnt[i];
-      cur_sel = ly.sel_idx ? ly.sel_idx : p.sel[i];
-      cur_sel_cnt = ly.sel_cnt ? ly.sel_cnt : p.sel_cnt[i];
-      int32_t r = csa2_index_full(ly.q, ly.w, &ly.keys, s->seq_of_query, s->query_pos, s->nq, s->H, s->D_idx,
-                                  s->max_ctx, nullptr, 0, s->P, cur_pool, cur_pool_cnt, s->K, cur_sel,
-                                  cur_sel_cnt, p.index_base, p.index_ws, status, stream);
-      if (r != CSA2_OK) return r;
-    } else if (modes[i] == CSA2_REINDEX) {
-      cur_sel = ly.sel_idx ? ly.sel_idx : p.sel[i];
-      cur_sel_cnt = ly.sel_cnt ? ly.sel_cnt : p.sel_cnt[i];
-      int32_t r = csa2_reindex(ly.q, ly.w, &ly.keys, s->seq_of_query, cur_pool, cur_pool_cnt, s->nq, s->H,
-                               s->D_idx, s->P, s->K, cur_sel, cur_sel_cnt, nullptr, p.reindex_base,
-                               p.reindex_ws, status, stream);
-      if (r != CSA2_OK) return r;
+      pool_of[i] = ly.pool_idx ? ly.pool_idx : p.pool[i];
+      pool_cnt_of[i] = ly.pool_cnt ? ly.pool_cnt : p.pool_cnt[i];
     } else {
-      // REUSE: the selection of the most recent FULL/REINDEX layer, unchanged.
-      if (ly.sel_idx && ly.sel_idx != cur_sel) {
-        if (cudaMemcpyAsync(ly.sel_idx, cur_sel, (size_t)s->nq * s->K * 4, cudaMemcpyDeviceToDevice, st) !=
+      pool_of[i] = pool_of[i - 1];
+      pool_cnt_of[i] = pool_cnt_of[i - 1];
+    }
+    if (modes[i] == CSA2_REUSE) {
+      sel_of[i] = sel_of[i - 1];
+      sel_cnt_of[i] = sel_cnt_of[i - 1];
+    } else {
+      sel_of[i] = ly.sel_idx ? ly.sel_idx : p.sel[i];
+      sel_cnt_of[i] = ly.sel_cnt ? ly.sel_cnt : p.sel_cnt[i];
+    }
+  }
+  // Every FULL layer, then in one launch the REINDEX layers that search its pool.
+  for (int i = 0; i < L; ++i) {
+    if (modes[i] != CSA2_FULL) continue;
+    const csa2_layer& ly = layers[i];
+    int32_t r = csa2_index_full(ly.q, ly.w, &ly.keys, s->seq_of_query, s->query_pos, s->nq, s->H, s->D_idx,
+                                s->max_ctx, nullptr, 0, s->P, pool_of[i], pool_cnt_of[i], s->K, sel_of[i],
+                                sel_cnt_of[i], p.index_base, p.index_ws, status, stream);
+    if (r != CSA2_OK) return r;
+    ReindexJobDesc rj[kMaxReindexJobs];
+    int n = 0;
+    for (int j = i + 1; j <= L; ++j) {
+      const bool end = j == L || modes[j] == CSA2_FULL;
+      if (!end && modes[j] == CSA2_REINDEX)
+        rj[n++] = ReindexJobDesc{layers[j].q, layers[j].w, &layers[j].keys, nullptr, sel_of[j], sel_cnt_of[j]};
+      if (n > 0 && (end || n == kMaxReindexJobs)) {
+        r = run_reindex(rj, n, s->seq_of_query, pool_of[i], pool_cnt_of[i], s->nq, s->H, s->D_idx, s->P, s->K,
+                        p.reindex_base, status, st);
+        if (r != CSA2_OK) return r;
+        n = 0;
+      }
+      if (end) break;
+    }
+  }
+  // REUSE layers with outputs of their own get a copy of the selection they use.
+  AttnJobDesc jobs[kMaxAttnJobs];
+  for (int i = 0; i < L; ++i) {
+    const csa2_layer& ly = layers[i];
+    if (modes[i] == CSA2_REUSE) {
+      if (ly.sel_idx && ly.sel_idx != sel_of[i]) {
+        if (cudaMemcpyAsync(ly.sel_idx, sel_of[i], (size_t)s->nq * s->K * 4, cudaMemcpyDeviceToDevice, st) !=
             cudaSuccess)
           return CSA2_ERR_CUDA;
       }
-      if (ly.sel_cnt && ly.sel_cnt != cur_sel_cnt) {
-        if (cudaMemcpyAsync(ly.sel_cnt, cur_sel_cnt, (size_t)s->nq * 4, cudaMemcpyDeviceToDevice, st) !=
+      if (ly.sel_cnt && ly.sel_cnt != sel_cnt_of[i]) {
+        if (cudaMemcpyAsync(ly.sel_cnt, sel_cnt_of[i], (size_t)s->nq * 4, cudaMemcpyDeviceToDevice, st) !=
             cudaSuccess)
           return CSA2_ERR_CUDA;
       }
     }
-    jobs[i] = AttnJobDesc{ly.q_attn, &ly.codes, &ly.scales, cur_sel, cur_sel_cnt, ly.out, ly.lse};
+    jobs[i] = AttnJobDesc{ly.q_attn, &ly.codes, &ly.scales, sel_of[i], sel_cnt_of[i], ly.out, ly.lse};
   }
   const float scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->D);
   return cuda_status(launch_sparse_attn_jobs(jobs, L, s->seq_of_query, s->query_pos, s->nq, s->Hq, s->D, s->K,

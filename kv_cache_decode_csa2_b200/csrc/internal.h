@@ -103,6 +103,35 @@ cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_ro
                                  const int32_t* pool_cnt, int32_t nq, int32_t H, int32_t D,
                                  int32_t P, int32_t* scores, int32_t* status, cudaStream_t st);
 
+// K3 fused: scores and top-K of up to kMaxReindexJobs reindex layers that
+// search the same pool, in one launch of co-resident CTAs.
+constexpr int kMaxReindexJobs = 8;
+struct ReindexJobDesc {
+  const int8_t* q;           // [nq][H][D]
+  const int8_t* w;           // [nq][H]
+  const csa2_rows* keys;
+  int32_t* scores;           // [nq][P] or nullptr
+  int32_t* sel_idx;          // [nq][K]
+  int32_t* sel_cnt;          // [nq] or nullptr
+};
+struct ReindexSelScratch {
+  int32_t n_probs;           // (layer, query) pairs it holds
+  uint32_t* hist;            // [n_probs][kBuckets], then hdr: zeroed by the launcher
+  uint32_t* hdr;             // [n_probs][4]
+  uint64_t* ties;
+  uint32_t* mcnt;
+  uint32_t* radix;
+};
+size_t reindex_select_scratch_bytes(int32_t n_probs, int32_t P);
+ReindexSelScratch carve_reindex_select(Carver& c, int32_t n_probs, int32_t P);
+// Returns cudaErrorNotSupported, having queued nothing, when the CTAs cannot
+// be co-resident or the head count is above 64; the caller then scores and
+// selects in separate launches.
+cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* seq_of_query,
+                                  const int32_t* pool_idx, const int32_t* pool_cnt, int32_t nq, int32_t H,
+                                  int32_t D, int32_t P, int32_t K, const ReindexSelScratch& r,
+                                  int32_t* status, cudaStream_t st);
+
 // K4: FP4 sparse attention.
 size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
 cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,

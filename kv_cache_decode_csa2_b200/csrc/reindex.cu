@@ -6,10 +6,20 @@
 // layer's index keys by position into a swizzled K-major tile (16-byte cp.async
 // per chunk: a pool row is one 128-byte line).  It runs one tcgen05 int8 MMA
 // group, D[128 slots x N heads] in TMEM, and applies the ReLU and head-weight
-// epilogue of the full-mode scorer.  The top-K then runs on these P scores in
-// shared memory (topk_small).
+// epilogue of the full-mode scorer.
+//
+// reindex_select_kernel goes on to the top-K of the layer in the same launch:
+// the CTAs of a pool (every CTA holds 128 of its scores, one per thread) are
+// co-resident and meet at bounded grid barriers.  They build the bucket
+// histogram of the pool in global memory, find the threshold bucket b*, rank
+// the ties at b* (the pool's tie list, staged in shared memory), and write the
+// members in slot order, which is position order because pool positions
+// ascend.  One launch serves every reindex layer that searches the same pool.
+// reindex_score_kernel alone (scores, then the select kernel) serves the
+// batches too large to be co-resident.
 #include "csa2_device.cuh"
 #include "internal.h"
+#include "select_common.cuh"
 
 namespace csa2 {
 
@@ -149,6 +159,327 @@ cudaError_t launch_r(const ReindexArgs& a, int nq, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+
+// ------------------------------------------------------------------ fused scoring + top-K
+constexpr int kRTieCap = 2048;   // ties of one pool ranked in shared memory (more: radix select)
+
+struct RSelJob {
+  const int8_t* q;
+  const int8_t* w;
+  const uint8_t* base;
+  int64_t row_bytes;
+  RowMap rows;
+  int32_t* scores;    // [nq][P] or nullptr
+  int32_t* sel_idx;   // [nq][K]
+  int32_t* sel_cnt;   // [nq] or nullptr
+};
+
+struct RSelArgs {
+  RSelJob job[kMaxReindexJobs];
+  const int32_t* seq_of_query;
+  const int32_t* pool_idx;
+  const int32_t* pool_cnt;
+  int32_t H, P, K, nq, G;
+  uint32_t* hist;     // [probs][kBuckets]   zeroed before the launch
+  uint32_t* hdr;      // [probs][4]          zeroed before the launch: barrier count, tie count
+  uint64_t* ties;     // [probs][kRTieCap]
+  uint32_t* mcnt;     // [probs][G]
+  uint32_t* radix;    // [probs][8][256]
+  int32_t* status;
+};
+
+// Dynamic shared memory: the T tiles of 128 pool rows and the query (then the
+// pool's ties), w, this CTA's ties, the MMA barrier and the TMEM address.
+template <int D, int N, int T>
+struct RSelLayout {
+  static constexpr int NT = 128 * T;
+  static constexpr size_t tiles = (size_t)(T * 128 * D + N * D);
+  static constexpr size_t region = tiles > (size_t)kRTieCap * 8 ? tiles : (size_t)kRTieCap * 8;
+  static constexpr size_t smem = 1024 + region + 128 * 4 + NT * 8 + 64;
+  static constexpr uint32_t cols = T * N <= 32 ? 32 : T * N <= 64 ? 64 : T * N <= 128 ? 128 : 256;
+};
+
+// T tiles of 128 pool slots per CTA (one slot per thread): the device holds
+// one such CTA per SM, so T sets how many pools fit in one launch.
+template <int D, int N, int T>
+__global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid_constant__ RSelArgs a) {
+  using Lay = RSelLayout<D, N, T>;
+  constexpr int NT = Lay::NT;
+  constexpr uint32_t TMEM_COLS = Lay::cols;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* atile = smem;                                   // T x 128 x D   (scoring)
+  uint8_t* bmat = atile + T * 128 * D;                     // N x D         (scoring)
+  uint64_t* rowties = reinterpret_cast<uint64_t*>(smem);   // the pool's ties (after scoring)
+  int32_t* w_s = reinterpret_cast<int32_t*>(smem + Lay::region);
+  uint64_t* own = reinterpret_cast<uint64_t*>(w_s + 128);  // this CTA's ties (at most NT)
+  uint64_t* bar = own + NT;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 1);
+  __shared__ uint64_t wtmp[NT / 32];
+  __shared__ int32_t bstar_s, above_s;
+  __shared__ uint32_t own_cnt, wcnt[NT / 32];
+  __shared__ unsigned long long kthr_s;
+  __shared__ RadixSmem rsm;
+
+  const int x = blockIdx.x, q = blockIdx.y, jb = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const RSelJob& J = a.job[jb];
+  const int prob = jb * a.nq + q;
+  const int G = a.G;
+  int32_t cnt = __ldg(a.pool_cnt + q);
+  cnt = cnt < 0 ? 0 : (cnt > a.P ? a.P : cnt);
+  const int32_t slot0 = x * NT, slot = slot0 + tid;
+  const bool has = slot0 < cnt;   // CTA-uniform: this CTA holds pool entries
+  const bool valid = slot < cnt;
+  const int32_t* pidx = a.pool_idx + (int64_t)q * a.P;
+  const int32_t pos = valid ? __ldg(pidx + slot) : -1;
+  const int32_t prev = (valid && slot > 0) ? __ldg(pidx + slot - 1) : INT32_MIN;
+  if (tid == 0) {
+    bstar_s = -1;
+    above_s = 0;
+    own_cnt = 0;
+    kthr_s = ~0ull;
+  }
+  if (valid && pos <= prev) record_error(a.status, CSA2_ERR_ORDER);   // pool positions ascend
+
+  // ---- scores of this CTA's NT pool entries (one per thread)
+  int32_t s = 0;
+  if (has) {
+    const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
+    if (warp == 0) {
+      tmem_alloc(tmem_slot, TMEM_COLS);
+      tmem_relinquish();
+    }
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      fence_mbar_init();
+    }
+    {
+      const uint8_t* src = nullptr;
+      if (valid) {
+        const int64_t row = pos >= 0 ? map_row(J.rows, seq, pos) : -1;
+        if (row < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+        else src = J.base + row * J.row_bytes;
+      }
+      uint8_t* tile = atile + (tid >> 7) * 128 * D;
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {
+        uint8_t* dst = tile + swizzled_chunk(tid & 127, c, D);
+        if (src) cp_async16(dst, src + 16 * c);
+        else *reinterpret_cast<int4*>(dst) = make_int4(0, 0, 0, 0);
+      }
+    }
+    const int8_t* qsrc = J.q + (int64_t)q * a.H * D;
+    for (int idx = tid; idx < N * (D / 16); idx += NT) {
+      const int r = idx / (D / 16), c = idx % (D / 16);
+      int4 v = make_int4(0, 0, 0, 0);
+      if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
+      *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
+    }
+    if (tid < N) w_s[tid] = tid < a.H ? (int32_t)__ldg(J.w + (int64_t)q * a.H + tid) : 0;
+    cp_async_wait_all();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    if (tid == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, N);
+      const uint32_t a_addr = smem_u32(atile), b_addr = smem_u32(bmat);
+#pragma unroll
+      for (int t = 0; t < T; ++t)   // tile t accumulates in TMEM columns [t N, t N + N)
+#pragma unroll
+        for (int k = 0; k < D / 32; ++k)
+          mma_i8(tmem_base + t * N, smem_desc_kmajor(a_addr + t * 128 * D + 32 * k, D),
+                 smem_desc_kmajor(b_addr + 32 * k, D), idesc, k > 0 ? 1u : 0u);
+      mma_commit(bar);
+    }
+    volatile int32_t never = 0;
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar, 0, &never));
+    if (ok) {
+      tc_fence_after();
+      // warp w reads TMEM lanes 32 (w % 4) .. (a warp's lane quarter) of tile w / 4
+      const uint32_t taddr = tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + (uint32_t)((warp >> 2) * N);
+      if constexpr (N == 16) {
+        uint32_t r16[16];
+        tmem_ld16(taddr, r16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 16; ++h) s += w_s[h] * max((int32_t)r16[h], 0);
+      } else {
+#pragma unroll 1
+        for (int g = 0; g < N / 32; ++g) {
+          uint32_t r32[32];
+          tmem_ld32(taddr + 32 * g, r32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int h = 0; h < 32; ++h) s += w_s[g * 32 + h] * max((int32_t)r32[h], 0);
+        }
+      }
+    } else if (tid == 0) {
+      record_error(a.status, CSA2_ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();   // also: the tiles are free for the tie list from here on
+    if (warp == 0) {
+      tc_fence_after();
+      tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+  }
+  if (J.scores && valid) J.scores[(int64_t)q * a.P + slot] = s;
+
+  // ---- the pool's bucket histogram, then the threshold bucket
+  uint32_t* hist = a.hist + (size_t)prob * kBuckets;
+  uint32_t* hdr = a.hdr + (size_t)prob * 4;
+  const int32_t bk = (int32_t)score_bucket(s);
+  if (valid) atomicAdd(&hist[bk], 1u);
+  uint32_t phase = 0;
+  sel_grid_sync(&hdr[0], ++phase * G, a.status);
+  constexpr int kBins = kBuckets / NT;   // bins per thread
+  uint4 hv[kBins / 4];
+  const uint4* hp = reinterpret_cast<const uint4*>(hist + tid * kBins);
+#pragma unroll
+  for (int u = 0; u < kBins / 4; ++u) hv[u] = __ldcg(hp + u);
+  uint32_t hsum = 0;
+#pragma unroll
+  for (int u = 0; u < kBins / 4; ++u) hsum += hv[u].x + hv[u].y + hv[u].z + hv[u].w;
+  uint64_t total64;
+  const uint64_t hex = sel_scan<NT>(hsum, wtmp, &total64);
+  const int64_t total = (int64_t)total64;
+  const int64_t above_me = total - (int64_t)hex - hsum;
+  const int32_t K = a.K;
+  if (total > K && above_me < K && above_me + hsum >= K) {
+    int64_t acc = above_me;
+    bool found = false;
+#pragma unroll
+    for (int u = kBins / 4 - 1; u >= 0; --u) {
+      const uint32_t v4[4] = {hv[u].x, hv[u].y, hv[u].z, hv[u].w};
+#pragma unroll
+      for (int e = 3; e >= 0; --e) {
+        if (!found && acc + v4[e] >= K) {
+          bstar_s = tid * kBins + 4 * u + e;
+          above_s = (int32_t)acc;
+          found = true;
+        }
+        if (!found) acc += v4[e];
+      }
+    }
+  }
+  __syncthreads();
+  const int32_t bstar = bstar_s;   // -1: every valid entry is a member
+
+  // ---- ties at b*: ranked against the pool's tie list
+  const uint64_t key = cand_key(s, slot);
+  const bool above = valid && bk > bstar;
+  const bool tie = valid && bk == bstar;
+  if (bstar >= 0) {
+    if (tie) {
+      own[atomicAdd(&own_cnt, 1u)] = key;
+      const uint32_t g = atomicAdd(&hdr[1], 1u);
+      if (g < (uint32_t)kRTieCap) a.ties[(size_t)prob * kRTieCap + g] = key;
+    }
+    sel_grid_sync(&hdr[0], ++phase * G, a.status);
+    const uint32_t nt = __ldcg(&hdr[1]);
+    const int32_t need = K - above_s;
+    if (nt <= (uint32_t)kRTieCap) {
+      const uint64_t* src = a.ties + (size_t)prob * kRTieCap;
+      for (uint32_t i = tid; i < nt; i += NT) rowties[i] = __ldcg(src + i);
+      __syncthreads();
+      for (uint32_t i = warp; i < own_cnt; i += NT / 32) {
+        const uint64_t ki = own[i];
+        uint32_t r = 0;
+#pragma unroll 4
+        for (uint32_t j = lane; j < nt; j += 32) r += rowties[j] > ki;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+        if (lane == 0 && (int32_t)r < need) atomicMin(&kthr_s, (unsigned long long)ki);
+      }
+    } else {
+      const int32_t sv[1] = {s};
+      const uint64_t kth = radix_kth<NT, 1>(sv, tie ? 1u : 0u, slot, need, G, x,
+                                             a.radix + (size_t)prob * 8 * 256, &hdr[0], phase, a.status, rsm);
+      if (tid == 0) kthr_s = kth;
+    }
+    __syncthreads();
+  }
+  const bool member = above || (tie && key >= kthr_s);
+
+  // ---- slots: within the CTA by ballot, across CTAs from the published counts
+  const uint32_t bal = __ballot_sync(0xffffffffu, member);
+  if (lane == 0) wcnt[warp] = __popc(bal);
+  __syncthreads();
+  uint32_t before = __popc(bal & ((1u << lane) - 1u)), cta_cnt = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    before += w < warp ? wcnt[w] : 0u;
+    cta_cnt += wcnt[w];
+  }
+  uint32_t* mc = a.mcnt + (size_t)prob * G;
+  if (tid == 0) mc[x] = cta_cnt;
+  sel_grid_sync(&hdr[0], ++phase * G, a.status);
+  uint64_t part = 0ull;   // (members of the CTAs before) | (all members) << 32
+  for (int r = tid; r < G; r += NT) {
+    const uint64_t v = __ldcg(mc + r);
+    part += (r < x ? v : 0ull) | (v << 32);
+  }
+  uint64_t sums;
+  sel_scan<NT>(part, wtmp, &sums);
+  const int64_t off = (int64_t)(sums & 0xffffffffu), grand = (int64_t)(sums >> 32);
+  int32_t* dst = J.sel_idx + (int64_t)q * K;
+  if (member && off + before < K) dst[off + before] = pos;
+  if (x == G - 1) {
+    const int32_t n_out = grand < K ? (int32_t)grand : K;
+    for (int32_t i = n_out + tid; i < K; i += NT) dst[i] = -1;
+    if (tid == 0 && J.sel_cnt) J.sel_cnt[q] = n_out;
+  }
+}
+
+template <int D, int N, int T>
+cudaError_t launch_rs_t(const RSelArgs& a_in, int n_jobs, int nq, size_t zero_bytes, cudaStream_t st) {
+  using Lay = RSelLayout<D, N, T>;
+  constexpr size_t smem = Lay::smem;
+  static unsigned long long done = 0;
+  static int max_ctas[64];
+  cudaError_t e = ensure_smem(reindex_select_kernel<D, N, T>, (int)smem, done);
+  if (e != cudaSuccess) return e;
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 64) return cudaErrorNotSupported;
+  if (!max_ctas[dev]) {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reindex_select_kernel<D, N, T>, Lay::NT, smem);
+    if (e != cudaSuccess) return e;
+    max_ctas[dev] = per_sm * sm_count();
+  }
+  RSelArgs a = a_in;
+  a.G = (a.P + Lay::NT - 1) / Lay::NT;
+  if ((int64_t)a.G * nq * n_jobs > max_ctas[dev]) return cudaErrorNotSupported;
+  e = cudaMemsetAsync(a.hist, 0, zero_bytes, st);   // histograms and barrier headers
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.G, nq, n_jobs);
+  cfg.blockDim = dim3(Lay::NT, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, reindex_select_kernel<D, N, T>, a);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// Two tiles per CTA when the CTAs fit on the device, else four.
+template <int D, int N>
+cudaError_t launch_rs(const RSelArgs& a, int n_jobs, int nq, size_t zero_bytes, cudaStream_t st) {
+  cudaError_t e = launch_rs_t<D, N, 2>(a, n_jobs, nq, zero_bytes, st);
+  if (e != cudaErrorNotSupported) return e;
+  return launch_rs_t<D, N, 4>(a, n_jobs, nq, zero_bytes, st);
+}
+
 }  // namespace
 
 cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
@@ -171,6 +502,66 @@ cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_ro
     case 32: return launch_r<64, 32>(a, nq, st);
     case 64: return launch_r<64, 64>(a, nq, st);
     default: return launch_r<64, 128>(a, nq, st);
+  }
+}
+
+size_t reindex_select_scratch_bytes(int32_t n_probs, int32_t P) {
+  Carver c(nullptr);
+  ReindexSelScratch r = carve_reindex_select(c, n_probs, P);
+  (void)r;
+  return c.used + 256;
+}
+
+ReindexSelScratch carve_reindex_select(Carver& c, int32_t n_probs, int32_t P) {
+  const int32_t G = (P + 255) / 256;   // CTAs per pool: at least 256 slots each
+  ReindexSelScratch r;
+  r.n_probs = n_probs;
+  r.hist = c.take<uint32_t>((size_t)n_probs * kBuckets);
+  r.hdr = c.take<uint32_t>((size_t)n_probs * 4);   // directly after hist: one memset zeroes both
+  r.ties = c.take<uint64_t>((size_t)n_probs * kRTieCap);
+  r.mcnt = c.take<uint32_t>((size_t)n_probs * G);
+  r.radix = c.take<uint32_t>((size_t)n_probs * 8 * 256);
+  return r;
+}
+
+cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* seq_of_query,
+                                  const int32_t* pool_idx, const int32_t* pool_cnt, int32_t nq, int32_t H,
+                                  int32_t D, int32_t P, int32_t K, const ReindexSelScratch& r,
+                                  int32_t* status, cudaStream_t st) {
+  if (n_jobs < 1 || n_jobs > kMaxReindexJobs || r.n_probs < n_jobs * nq) return cudaErrorInvalidValue;
+  RSelArgs a{};
+  for (int j = 0; j < n_jobs; ++j) {
+    const ReindexJobDesc& d = jobs[j];
+    a.job[j] = RSelJob{d.q, d.w, static_cast<const uint8_t*>(d.keys->base), d.keys->row_bytes, to_rowmap(*d.keys),
+                       d.scores, d.sel_idx, d.sel_cnt};
+  }
+  a.seq_of_query = seq_of_query;
+  a.pool_idx = pool_idx;
+  a.pool_cnt = pool_cnt;
+  a.H = H;
+  a.P = P;
+  a.K = K;
+  a.nq = nq;
+  a.hist = r.hist;
+  a.hdr = r.hdr;
+  a.ties = r.ties;
+  a.mcnt = r.mcnt;
+  a.radix = r.radix;
+  a.status = status;
+  const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
+  if (N == 128) return cudaErrorNotSupported;
+  const size_t zb = (size_t)n_jobs * nq * (kBuckets + 4) * sizeof(uint32_t);
+  if (D == 128) {
+    switch (N) {
+      case 16: return launch_rs<128, 16>(a, n_jobs, nq, zb, st);
+      case 32: return launch_rs<128, 32>(a, n_jobs, nq, zb, st);
+      default: return launch_rs<128, 64>(a, n_jobs, nq, zb, st);
+    }
+  }
+  switch (N) {
+    case 16: return launch_rs<64, 16>(a, n_jobs, nq, zb, st);
+    case 32: return launch_rs<64, 32>(a, n_jobs, nq, zb, st);
+    default: return launch_rs<64, 64>(a, n_jobs, nq, zb, st);
   }
 }
 

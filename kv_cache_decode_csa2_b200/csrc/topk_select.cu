@@ -26,6 +26,7 @@
 // of the 64-bit key per pass.
 #include "csa2_device.cuh"
 #include "internal.h"
+#include "select_common.cuh"
 
 namespace csa2 {
 
@@ -72,58 +73,6 @@ __device__ __forceinline__ int32_t sel_n(const SelArgs& a, int q) {
   return a.n_max;
 }
 
-// Exclusive block scan of kSelNT values (pairs of 32-bit counts packed in 64
-// bits add without carries); *total gets the sum.  Ends with a barrier, so
-// wtmp can be reused at once.
-__device__ __forceinline__ uint64_t sel_scan(uint64_t v, uint64_t* wtmp, uint64_t* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) wtmp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    uint64_t y = wtmp[lane];
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint64_t z = __shfl_up_sync(0xffffffffu, y, o);
-      if (lane >= o) y += z;
-    }
-    wtmp[lane] = y;
-  }
-  __syncthreads();
-  const uint64_t base = warp > 0 ? wtmp[warp - 1] : 0ull;
-  *total = wtmp[31];
-  __syncthreads();
-  return base + x - v;
-}
-
-// Grid barrier of the G CTAs of one row: arrival count `target` (a multiple
-// of G).  Bounded: after kWaitLimitNs it records CSA2_ERR_TIMEOUT and goes on.
-__device__ __forceinline__ void sel_grid_sync(uint32_t* bar, uint32_t target, int32_t* status) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(bar, 1u);
-    const uint64_t t0 = global_ns();
-    while (true) {
-      uint32_t v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-      if (v >= target) break;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        record_error(status, CSA2_ERR_TIMEOUT);
-        break;
-      }
-      __nanosleep(32);
-    }
-    __threadfence();
-  }
-  __syncthreads();
-}
-
 // E candidates per thread (contiguous), kSelNT * E per CTA.
 template <int E>
 __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant__ SelArgs a) {
@@ -137,9 +86,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
   __shared__ int32_t bstar_s[2], above_s[2];
   __shared__ uint32_t own_cnt[2], gbase_s[2], nt_s[2];
   __shared__ unsigned long long kthr_s[2];
-  __shared__ uint32_t dig[256];
-  __shared__ unsigned long long prefix_s;
-  __shared__ int32_t rem_s;
+  __shared__ RadixSmem rsm;
   __shared__ uint64_t off_s, grand_s;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -215,7 +162,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
 #pragma unroll
   for (int b = 0; b < kBinsPer; ++b) hsum += hb[b];
   uint64_t total64;
-  const uint64_t excl = sel_scan(hsum, wtmp, &total64);
+  const uint64_t excl = sel_scan<kSelNT>(hsum, wtmp, &total64);
   const int64_t total = (int64_t)total64;
   const int64_t above_me = total - (int64_t)excl - hsum;   // candidates in the bins above this thread's
 #pragma unroll
@@ -308,66 +255,9 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
   for (int t = 0; t < 2; ++t) {
     if (bstar_s[t] < 0 || nt[t] <= (uint32_t)kSelTieCap) continue;
     uint32_t* gbins = G > 1 ? a.radix + ((size_t)q * 2 + t) * 8 * 256 : nullptr;
-    if (G > 1) {
-      if (c == 0)
-        for (int i = tid; i < 8 * 256; i += kSelNT) gbins[i] = 0u;
-      sel_grid_sync(&hdr[0], ++phase * G, a.status);
-    }
-    const uint32_t tm = t ? tie_m[1] : tie_m[0];
-    uint64_t prefix = 0ull, fixed = 0ull;
-    int32_t rem = a.k[t] - above_s[t];
-    for (int pass = 0; pass < 8; ++pass) {
-      const int shift = 56 - 8 * pass;
-      if (tid < 256) dig[tid] = 0u;
-      __syncthreads();
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        if ((tm >> i) & 1u) {
-          const uint64_t key = cand_key(s[i], j0 + i);
-          if ((key & fixed) == prefix) atomicAdd(&dig[(key >> shift) & 255u], 1u);
-        }
-      }
-      __syncthreads();
-      if (G > 1) {
-        if (tid < 256 && dig[tid]) atomicAdd(&gbins[pass * 256 + tid], dig[tid]);
-        sel_grid_sync(&hdr[0], ++phase * G, a.status);
-        if (tid < 256) dig[tid] = __ldcg(&gbins[pass * 256 + tid]);
-        __syncthreads();
-      }
-      if (warp == 0) {   // lane l holds digits 255-8l .. 248-8l (lane 0: the highest)
-        uint32_t d8[8], sum = 0;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          d8[u] = dig[255 - 8 * lane - u];
-          sum += d8[u];
-        }
-        uint32_t incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-          if (lane >= o) incl += y;
-        }
-        const uint32_t before = incl - sum;
-        if ((int64_t)before < rem && (int64_t)incl >= rem) {
-          uint32_t acc = before;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            if ((int64_t)acc + d8[u] >= rem) {
-              prefix_s = prefix | ((uint64_t)(255 - 8 * lane - u) << shift);
-              rem_s = rem - (int32_t)acc;
-              break;
-            }
-            acc += d8[u];
-          }
-        }
-      }
-      __syncthreads();
-      prefix = prefix_s;
-      rem = rem_s;
-      fixed |= 255ull << shift;
-      __syncthreads();
-    }
-    if (tid == 0) kthr_s[t] = prefix;
+    const uint64_t kth = radix_kth<kSelNT, E>(s, t ? tie_m[1] : tie_m[0], j0, a.k[t] - above_s[t], G, c, gbins,
+                                              hdr ? &hdr[0] : nullptr, phase, a.status, rsm);
+    if (tid == 0) kthr_s[t] = kth;
   }
   __syncthreads();
 
@@ -385,7 +275,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
   if (n_k < 2) mem[1] = 0u;
   const uint64_t pack = (uint64_t)__popc(mem[0]) | ((uint64_t)__popc(mem[1]) << 32);
   uint64_t cta_tot;
-  const uint64_t mexcl = sel_scan(pack, wtmp, &cta_tot);
+  const uint64_t mexcl = sel_scan<kSelNT>(pack, wtmp, &cta_tot);
   uint64_t off = 0ull, grand = cta_tot;
   if (G > 1) {
     uint32_t* mc = a.mcnt + (size_t)q * 2 * kSelMaxG;

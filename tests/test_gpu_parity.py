@@ -205,6 +205,46 @@ def test_reindex_matches_oracle(pool):
     assert np.array_equal(_np(re.sel_idx)[0], ref_sel) and int(_np(re.sel_cnt)[0]) == len(ref_sel)
 
 
+def test_reindex_flat_scores():
+    """All-zero reindex keys: every pool entry scores 0, so the top-K is the K
+    lowest pool positions (ties go to the lower position) and the tie list is
+    far longer than the ranked one: the radix select decides."""
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(40000,), modes=(synth.FULL, synth.REINDEX))
+    c = G.build(wl)
+    full, re = c.layers_dev
+    re.keys.data.zero_()
+    B.check_status(B.csa2_index_full(full.q, full.w, full.keys, c.pos_dev, c.max_ctx, P=wl.pool,
+                                     pool_idx=full.pool_idx, pool_cnt=full.pool_cnt))
+    B.check_status(B.csa2_reindex(re.q, re.w, re.keys, full.pool_idx, full.pool_cnt, wl.topk, re.sel_idx,
+                                  sel_cnt=re.sel_cnt))
+    q1, w1 = c.host_q[(1, 0)]
+    pool = _np(full.pool_idx)[0]
+    _, ref_sel = O.reindex(q1, w1, np.zeros_like(c.host_keys[(1, 0)]), pool, wl.topk)
+    assert np.array_equal(ref_sel, pool[:wl.topk])
+    assert np.array_equal(_np(re.sel_idx)[0], ref_sel) and int(_np(re.sel_cnt)[0]) == wl.topk
+
+
+def test_reindex_batch_of_many_queries():
+    """Eight queries of a 16384-entry pool: more CTAs than fit on the device at
+    once, so scoring and selection run as separate launches."""
+    wl = synth.scaled(synth.C3_RAGGED, ragged=(8, 17000, 30000), modes=(synth.FULL, synth.REINDEX), page_rows=0)
+    c = G.build(wl)
+    full, re = c.layers_dev
+    B.check_status(B.csa2_index_full(full.q, full.w, full.keys, c.pos_dev, c.max_ctx, P=wl.pool,
+                                     pool_idx=full.pool_idx, pool_cnt=full.pool_cnt, seq_of_query=c.seq_dev))
+    B.check_status(B.csa2_reindex(re.q, re.w, re.keys, full.pool_idx, full.pool_cnt, wl.topk, re.sel_idx,
+                                  sel_cnt=re.sel_cnt, seq_of_query=c.seq_dev))
+    pools, sels = _np(full.pool_idx), _np(re.sel_idx)
+    for i in range(len(c.query_pos)):
+        s = int(c.seq_of_query[i])
+        q0, w0 = c.host_q[(0, i)]
+        _, ref_pool, _ = O.full_index(q0, w0, c.host_keys[(0, s)], int(c.query_pos[i]), wl.pool, wl.topk)
+        q1, w1 = c.host_q[(1, i)]
+        _, ref_sel = O.reindex(q1, w1, c.host_keys[(1, s)], ref_pool, wl.topk)
+        assert np.array_equal(pools[i, :len(ref_pool)], ref_pool)
+        assert np.array_equal(sels[i, :len(ref_sel)], ref_sel)
+
+
 # ------------------------------------------------------------------ K4 attention
 @pytest.mark.parametrize("wl", [synth.C0_TINY, synth.scaled(synth.C1_SINGLE, seq_lens=(3001,))],
                          ids=["hq8_d128", "hq64_d512"])

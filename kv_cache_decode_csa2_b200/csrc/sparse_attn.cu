@@ -7,27 +7,33 @@
 // ascending, S is the selection entries below the window start, followed by
 // the window itself, and row j of S has a closed form.
 //
-// One CTA handles 64 rows of S for up to 64 query heads of one (layer,
-// query).  It gathers each row's E2M1 codes and E4M3 scales by position and
-// dequantises them exactly into bf16 in shared memory (a value with 2
-// significant bits times a scale with 4 significant bits fits bf16's 8 bits).
-// Then it computes logits = Q K^T and the unnormalised P V on bf16 tensor
-// cores with fp32 accumulation, and writes a (max, sum, O) partial per head.
-// A combine kernel merges the partials of every (layer, query, head).
-// Several layers of a plan go into one launch (a job array), so independent
-// layers run side by side.
+// A group of kCl CTAs handles one (layer, query, group of up to 32 heads).
+// CTA r of the group takes slice r of the selection entries (entries at or
+// above the window start are left to the window) and slice r of the window,
+// so no CTA waits for a count of the others.  It gathers each
+// row's E2M1 codes and E4M3 scales by position and dequantises them exactly
+// into bf16 in shared memory (a value with 2 significant bits times a scale
+// with 4 significant bits fits bf16's 8 bits).  Then it computes logits =
+// Q K^T and the unnormalised P V on bf16 tensor cores with fp32 accumulation,
+// tile by tile with an online softmax, and writes its partial (max, sum, O)
+// per head to L2.  When all CTAs of the launch fit on the device at once
+// (cooperative launch), the group meets at a bounded barrier and CTA r merges
+// columns [r D / kCl, (r + 1) D / kCl) of every head; otherwise a merge kernel
+// does the same.  Several layers of a plan go into one launch (a job array),
+// so independent layers run side by side.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include "csa2_device.cuh"
 #include "internal.h"
+#include "select_common.cuh"
 
 namespace csa2 {
 
 namespace {
 
-constexpr int kRows = 64;        // rows of S per CTA
-constexpr int kSelCache = 1024;  // selection entries kept in shared memory per CTA
+constexpr int kCl = 8;       // CTAs per group: row slices of one (layer, query, head group)
+constexpr int kTile = 80;    // rows of S per tile (a multiple of 16)
 constexpr int kMaxJobs = kMaxAttnJobs;
 
 struct AttnJob {
@@ -42,16 +48,18 @@ struct AttnJob {
   const int32_t* sel_cnt;
   uint16_t* out;
   float* lse;
-  float* part_o;     // [nq][Hq][n_chunks][D]
-  float* part_ml;    // [nq][Hq][n_chunks][2]
 };
 
 struct AttnArgs {
   AttnJob jobs[kMaxJobs];
   const int32_t* seq_of_query;
   const int32_t* query_pos;
-  int32_t nq, Hq, K, window, n_chunks, n_jobs;
+  int32_t nq, Hq, K, window, n_jobs;
   float scale_log2;
+  float* part_o;      // [groups][kCl][HG][D]   partial O of every CTA
+  float2* part_ml;    // [groups][kCl][HG]      its (max in log2 units, sum)
+  uint32_t* bar;      // [groups]               barrier counts (zeroed before a fused launch)
+  int32_t fused;      // the group merges in the same launch
   int32_t* status;
 };
 
@@ -110,343 +118,408 @@ template <int D, int HG>
 struct AttnSmem {
   static constexpr int kKV = 2 * D + 16;           // bytes per K/V row (padded against bank conflicts)
   static constexpr int kQ = 2 * D + 16;            // bytes per Q row
-  static constexpr int kP = 2 * kRows + 16;        // bytes per P row (bf16)
-  static constexpr int kS = kRows + 4;             // floats per logit row
-  static constexpr size_t kv = 0;
-  static constexpr size_t qo = kv + (size_t)kRows * kKV;
+  static constexpr int kP = 2 * kTile + 16;        // bytes per P row (bf16)
+  static constexpr int kS = kTile + 4;             // floats per logit row
+  static constexpr size_t kv = 0;                  // K/V tile; at the end the partial O [HG][D] fp32
+  static constexpr size_t qo = kv + (size_t)kTile * kKV;
   static constexpr size_t po = qo + (size_t)HG * kQ;
   static constexpr size_t so = po + (size_t)HG * kP;
-  static constexpr size_t mo = so + (size_t)HG * kS * 4;
-  static constexpr size_t pos_o = mo + (size_t)HG * 8;
-  static constexpr size_t row_o = pos_o + kRows * 4;
-  static constexpr size_t sel_o = row_o + 2 * kRows * 8;
-  static constexpr size_t total = sel_o + kSelCache * 4 + 64;
+  static constexpr size_t mo = so + (size_t)HG * kS * 4;    // [HG][4]: max (log2 units), sum, rescale
+  static constexpr size_t pos_o = mo + (size_t)HG * 16;
+  static constexpr size_t row_o = pos_o + kTile * 4;
+  static constexpr size_t total = row_o + 2 * kTile * 8 + 64;
+  static_assert((size_t)(3 * kCl + 2) * HG * 4 <= (size_t)HG * kS * 4, "merge tables fit in the logits");
 };
 
-template <int D, int HG>
-__global__ void __launch_bounds__(256, 1) sparse_attn_kernel(const __grid_constant__ AttnArgs a) {
+// Merges the kCl partials of group gidx for columns [r CW, r CW + CW) of
+// every head: per head the overall max M, the denominator L and the weight
+// 2^(m_c - M) / L of every CTA c, then float4 items of the weighted sum.
+template <int D, int HG, int NTHR>
+__device__ __forceinline__ void merge_slice(const AttnArgs& a, const AttnJob& J, int q, int h0, int gidx, int r,
+                                            float* tab) {
+  const int tid = threadIdx.x;
+  float* mtab = tab;                  // [kCl][HG]
+  float* ltab = mtab + kCl * HG;      // [kCl][HG]
+  float* ftab = ltab + kCl * HG;      // [kCl][HG]
+  float* Mh = ftab + kCl * HG;        // [HG]
+  float* Lh = Mh + HG;                // [HG]
+  const float2* pml = a.part_ml + (size_t)gidx * kCl * HG;
+  for (int i = tid; i < kCl * HG; i += NTHR) {
+    const float2 ml = __ldcg(pml + i);
+    mtab[i] = ml.x;
+    ltab[i] = ml.y;
+  }
+  __syncthreads();
+  if (tid < HG) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < kCl; ++c) M = fmaxf(M, mtab[c * HG + tid]);
+    float Ls = 0.f;
+#pragma unroll
+    for (int c = 0; c < kCl; ++c) {
+      const float mc = mtab[c * HG + tid];
+      if (mc != -INFINITY) Ls += exp2f(mc - M) * ltab[c * HG + tid];
+    }
+    const float inv = Ls > 0.f ? 1.f / Ls : 0.f;
+#pragma unroll
+    for (int c = 0; c < kCl; ++c) {
+      const float mc = mtab[c * HG + tid];
+      ftab[c * HG + tid] = mc == -INFINITY ? 0.f : exp2f(mc - M) * inv;
+    }
+    Mh[tid] = M;
+    Lh[tid] = Ls;
+  }
+  __syncthreads();
+  constexpr int CW = D / kCl;
+  constexpr int C4 = CW / 4;
+  constexpr int F4 = HG * C4;
+  const float* po = a.part_o + (size_t)gidx * kCl * HG * D;
+  for (int f = tid; f < F4; f += NTHR) {
+    const int h = f / C4, col = r * CW + (f % C4) * 4;
+    float4 v[kCl];
+#pragma unroll
+    for (int c = 0; c < kCl; ++c)
+      v[c] = __ldcg(reinterpret_cast<const float4*>(po + ((size_t)c * HG + h) * D + col));
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int c = 0; c < kCl; ++c) {
+      const float w = ftab[c * HG + h];
+      o.x += w * v[c].x;
+      o.y += w * v[c].y;
+      o.z += w * v[c].z;
+      o.w += w * v[c].w;
+    }
+    if (h0 + h < a.Hq) {
+      const __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y), hi = __floats2bfloat162_rn(o.z, o.w);
+      uint2 pk;
+      pk.x = *reinterpret_cast<const uint32_t*>(&lo);
+      pk.y = *reinterpret_cast<const uint32_t*>(&hi);
+      *reinterpret_cast<uint2*>(J.out + ((size_t)q * a.Hq + h0 + h) * D + col) = pk;
+    }
+  }
+  if (r == 0 && tid < HG && h0 + tid < a.Hq && J.lse)
+    J.lse[(size_t)q * a.Hq + h0 + tid] = (Mh[tid] + log2f(Lh[tid])) * 0.69314718055994531f;
+}
+
+template <int D, int HG, int NTHR>
+__global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_constant__ AttnArgs a) {
   using L = AttnSmem<D, HG>;
-  constexpr int NM = HG / 16;          // m-tiles (16 heads each)
-  constexpr int WPM = 8 / NM;          // warps per m-tile
-  constexpr int NT_S = 8 / WPM;        // 8-row n-tiles of logits per warp
-  constexpr int DW = D / WPM;          // output columns per warp
-  constexpr int NT_O = DW / 8;         // 8-column n-tiles of output per warp
+  constexpr int NW = NTHR / 32;                      // warps
+  constexpr int NM = HG / 16;                        // m-tiles (16 heads each)
+  constexpr int WPM = NW / NM;                       // warps per m-tile
+  constexpr int NTS = kTile / 8;                     // 8-row n-tiles of logits per tile
+  constexpr int NTS_W = (NTS + WPM - 1) / WPM;       // of them per warp (at most)
+  constexpr int DW = D / WPM;                        // output columns per warp
+  constexpr int NT_O = DW / 8;                       // 8-column n-tiles of output per warp
+  constexpr int TPH = NTHR / HG;                     // softmax threads per head
+  constexpr int RPT = kTile / TPH;                   // rows per softmax thread
+  static_assert(kTile % 16 == 0 && kTile % TPH == 0 && NT_O % 2 == 0 && TPH <= 32, "tile shapes");
   extern __shared__ __align__(16) uint8_t sm[];
   uint8_t* kv_s = sm + L::kv;
   uint8_t* q_s = sm + L::qo;
   uint8_t* p_s = sm + L::po;
   float* s_s = reinterpret_cast<float*>(sm + L::so);
-  float* ml_s = reinterpret_cast<float*>(sm + L::mo);     // [HG][2]: running max (log2 units), sum
+  float* ml_s = reinterpret_cast<float*>(sm + L::mo);
   int32_t* pos_s = reinterpret_cast<int32_t*>(sm + L::pos_o);
-  int64_t* row_s = reinterpret_cast<int64_t*>(sm + L::row_o);     // [2][kRows]: code row, scale row
-  int32_t* sel_s = reinterpret_cast<int32_t*>(sm + L::sel_o);     // first kSelCache selection entries
-  __shared__ int32_t meta[4];
+  int64_t* row_s = reinterpret_cast<int64_t*>(sm + L::row_o);     // [2][kTile]: code row, scale row
 
+  const int rank = blockIdx.x;
+  const int gidx = blockIdx.z * gridDim.y + blockIdx.y;   // (job, query, head group)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int chunk = blockIdx.x, hg = blockIdx.y;
+  const int hg = blockIdx.y;
   const int job_i = blockIdx.z / a.nq, q = blockIdx.z % a.nq;
   const AttnJob& J = a.jobs[job_i];
   const int h0 = hg * HG;
 
-  // ---- Every load that does not depend on another is issued first: the Q
-  // rows of this head group, the query position and the selection count.
-  constexpr int QPER = HG * (D / 8) / 256;
+  // ---- independent loads first: Q rows of this head group, position, count
+  constexpr int QPER = HG * (D / 8) / NTHR;
+  static_assert(HG * (D / 8) % NTHR == 0, "whole Q items per thread");
   int4 qv[QPER];
 #pragma unroll
   for (int i = 0; i < QPER; ++i) {
-    const int idx = tid + i * 256, h = idx / (D / 8), c = idx % (D / 8);
+    const int idx = tid + i * NTHR, h = idx / (D / 8), c = idx % (D / 8);
     qv[i] = h0 + h < a.Hq ? __ldg(reinterpret_cast<const int4*>(J.q + ((size_t)q * a.Hq + h0 + h) * D) + c)
                           : make_int4(0, 0, 0, 0);
   }
   const int32_t pos = __ldg(a.query_pos + q);
   int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
-  if (tid == 0) meta[2] = 0;
+  const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
 #pragma unroll
   for (int i = 0; i < QPER; ++i) {
-    const int idx = tid + i * 256, h = idx / (D / 8), c = idx % (D / 8);
+    const int idx = tid + i * NTHR, h = idx / (D / 8), c = idx % (D / 8);
     *reinterpret_cast<int4*>(q_s + h * L::kQ + c * 16) = qv[i];
   }
-  // ---- S = (selection entries below the window start) followed by the window.
-  // The selection is ascending, so those entries are a prefix of it.  Count
-  // them in parallel, keeping the first kSelCache entries in shared memory
-  // for the row positions below.
+  if (tid < HG) {
+    ml_s[tid * 4 + 0] = -INFINITY;
+    ml_s[tid * 4 + 1] = 0.f;
+  }
+  if (tid == 0 && rank == 0 && pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+
+  // ---- this CTA's rows: selection entries [e0, e1) below the window start,
+  // then window offsets [o0, o1)
   cnt = cnt < 0 ? 0 : (cnt > a.K ? a.K : cnt);
   const int32_t wstart = pos - a.window + 1 > 0 ? pos - a.window + 1 : 0;
-  __syncthreads();
-  {
-    const int32_t* sel = J.sel_idx + (int64_t)q * a.K;
-    int32_t below = 0;
-    for (int base = 0; base < cnt; base += 4 * 256) {
-      int32_t v[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + u * 256 + tid;
-        v[u] = i < cnt ? __ldg(sel + i) : 0x7fffffff;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = base + u * 256 + tid;
-        below += v[u] < wstart;
-        if (i < kSelCache) sel_s[i] = v[u];
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) below += __shfl_xor_sync(0xffffffffu, below, o);
-    if (lane == 0 && below) atomicAdd(&meta[2], below);
-  }
-  if (tid == 0 && pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
-  __syncthreads();
-  const int32_t nsel = meta[2];
-  const int32_t nS = pos >= 0 ? nsel + (pos - wstart + 1) : 0;
-  const int32_t r0 = chunk * kRows;
-  const int nrows = nS - r0 < kRows ? nS - r0 : kRows;
-  const size_t pidx = ((size_t)q * a.Hq) * a.n_chunks + chunk;   // + h * n_chunks
-  if (nrows <= 0) {
-    for (int h = tid; h < HG && h0 + h < a.Hq; h += blockDim.x) {
-      float* ml = J.part_ml + (pidx + (size_t)(h0 + h) * a.n_chunks) * 2;
-      ml[0] = -INFINITY;
-      ml[1] = 0.f;
-    }
-    return;
-  }
-  const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
+  const int32_t wlen = pos >= 0 ? pos - wstart + 1 : 0;
+  const int32_t Ks = (a.K + kCl - 1) / kCl, Ws = (a.window + kCl - 1) / kCl;
+  const int32_t e0 = rank * Ks, o0 = rank * Ws;
+  const int32_t ns = (e0 + Ks < cnt ? e0 + Ks : cnt) - e0 > 0 ? (e0 + Ks < cnt ? e0 + Ks : cnt) - e0 : 0;
+  const int32_t nw = (o0 + Ws < wlen ? o0 + Ws : wlen) - o0 > 0 ? (o0 + Ws < wlen ? o0 + Ws : wlen) - o0 : 0;
+  const int32_t nrows = ns + nw;
+  const int32_t* sel = J.sel_idx + (int64_t)q * a.K + e0;
 
-  // ---- positions and physical rows of this chunk's rows
-  if (tid < kRows) {
-    int32_t p = -1;
-    int64_t cr = -1, sr = -1;
-    const int j = r0 + tid;
-    if (tid < nrows) {
-      p = j < nsel ? (j < kSelCache ? sel_s[j] : __ldg(J.sel_idx + (int64_t)q * a.K + j)) : wstart + (j - nsel);
-      if (p < 0 || p > pos) {
-        record_error(a.status, CSA2_ERR_INDEX_RANGE);
-        p = -1;
-      }
-    }
-    if (p >= 0) {
-      cr = map_row(J.cmap, seq, p);
-      sr = map_row(J.smap, seq, p);
-      if (cr < 0 || sr < 0) {
-        record_error(a.status, CSA2_ERR_INDEX_RANGE);
-        p = -1;
-        cr = sr = -1;
-      }
-    }
-    pos_s[tid] = p;
-    row_s[tid] = cr;
-    row_s[kRows + tid] = sr;
-  }
-  __syncthreads();
-  // ---- gather + dequantise: one (row, 8-element group) per item, so a warp
-  // reads 128 consecutive code bytes of a row and writes 512 consecutive bytes
-  // of shared memory (no bank conflicts).  All code words and scales of a
-  // thread are loaded before any is used.
-  {
-    constexpr int DPER = kRows * (D / 8) / 256;
-    uint32_t cw[DPER];
-    uint32_t sb[DPER];
+  float acc[NT_O][4];
 #pragma unroll
-    for (int u = 0; u < DPER; ++u) {
-      const int i = tid + u * 256, r = i / (D / 8), g = i % (D / 8);
-      const int64_t cr = row_s[r], sr = row_s[kRows + r];
-      cw[u] = cr >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(J.codes + cr * J.codes_rb) + g) : 0u;
-      sb[u] = cr >= 0 ? (uint32_t)__ldg(J.scales + sr * J.scales_rb + g / 4) : 0u;
-    }
-#pragma unroll
-    for (int u = 0; u < DPER; ++u) {
-      const int i = tid + u * 256, r = i / (D / 8), g = i % (D / 8);
-      uint32_t packed[4];
-      dequant8(cw[u], sb[u], packed);
-      *reinterpret_cast<uint4*>(kv_s + r * L::kKV + g * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-    }
-  }
-  __syncthreads();
+  for (int n = 0; n < NT_O; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+  const int mt = warp / WPM, wj = warp % WPM;
 
-  // ---- logits: S[h][r] = Q[h] . KV[r]  (tensor cores, fp32 accumulate)
-  {
-    const int mt = warp / WPM, nt0 = (warp % WPM) * NT_S;
-    float acc[NT_S][4];
+  for (int32_t t0 = 0; t0 < nrows; t0 += kTile) {
+    const int32_t tr = nrows - t0 < kTile ? nrows - t0 : kTile;
+    // ---- positions and physical rows of this tile
+    if (tid < kTile) {
+      int32_t p = -1;
+      int64_t cr = -1, sr = -1;
+      const int32_t r = t0 + tid;
+      if (tid < tr) {
+        if (r < ns) {
+          p = __ldg(sel + r);
+          if (p < 0 || p > pos) {
+            record_error(a.status, CSA2_ERR_INDEX_RANGE);
+            p = -1;
+          } else if (p >= wstart) {
+            p = -1;   // inside the window: counted there
+          }
+        } else {
+          p = wstart + o0 + (r - ns);
+        }
+      }
+      if (p >= 0) {
+        cr = map_row(J.cmap, seq, p);
+        sr = map_row(J.smap, seq, p);
+        if (cr < 0 || sr < 0) {
+          record_error(a.status, CSA2_ERR_INDEX_RANGE);
+          p = -1;
+          cr = sr = -1;
+        }
+      }
+      pos_s[tid] = p;
+      row_s[tid] = cr;
+      row_s[kTile + tid] = sr;
+    }
+    __syncthreads();
+    // ---- gather + dequantise: one (row, 8-element group) per item, so a warp
+    // reads 128 consecutive code bytes of a row and writes 512 consecutive
+    // bytes of shared memory.  All loads of a thread are issued before any use.
+    {
+      constexpr int DPER = kTile * (D / 8) / NTHR;
+      static_assert(kTile * (D / 8) % NTHR == 0, "whole items per thread");
+      uint32_t cw[DPER];
+      uint32_t sb[DPER];
 #pragma unroll
-    for (int n = 0; n < NT_S; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    const uint32_t qa = smem_u32(q_s + (mt * 16 + (lane & 15)) * L::kQ + (lane >> 4) * 16);
+      for (int u = 0; u < DPER; ++u) {
+        const int i = tid + u * NTHR, r = i / (D / 8), g = i % (D / 8);
+        const int64_t cr = row_s[r], sr = row_s[kTile + r];
+        cw[u] = cr >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(J.codes + cr * J.codes_rb) + g) : 0u;
+        sb[u] = cr >= 0 ? (uint32_t)__ldg(J.scales + sr * J.scales_rb + g / 4) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < DPER; ++u) {
+        const int i = tid + u * NTHR, r = i / (D / 8), g = i % (D / 8);
+        uint32_t packed[4];
+        dequant8(cw[u], sb[u], packed);
+        *reinterpret_cast<uint4*>(kv_s + r * L::kKV + g * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+    }
+    __syncthreads();
+    // ---- logits: S[h][r] = Q[h] . KV[r]
+    {
+      // with registers to spare, two accumulators per n-tile (even and odd k)
+      // halve the dependent MMA chain
+      constexpr int NACC = NTHR <= 256 ? 2 : 1;
+      float sacc[2][NTS_W][4];
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int n = 0; n < NTS_W; ++n) sacc[e][n][0] = sacc[e][n][1] = sacc[e][n][2] = sacc[e][n][3] = 0.f;
+      const uint32_t qa = smem_u32(q_s + (mt * 16 + (lane & 15)) * L::kQ + (lane >> 4) * 16);
 #pragma unroll 4
-    for (int k = 0; k < D / 16; ++k) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(qa + k * 32, a0, a1, a2, a3);
+      for (int k = 0; k < D / 16; ++k) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(qa + k * 32, a0, a1, a2, a3);
 #pragma unroll
-      for (int n = 0; n < NT_S; ++n) {
-        uint32_t b0, b1;
-        const int row = (nt0 + n) * 8 + (lane & 7);
-        ldsm_x2(smem_u32(kv_s + row * L::kKV + ((lane >> 3) & 1) * 16 + k * 32), b0, b1);
-        mma16816(acc[n], a0, a1, a2, a3, b0, b1);
+        for (int n = 0; n < NTS_W; ++n) {
+          const int nt = wj + n * WPM;
+          if (nt < NTS) {
+            uint32_t b0, b1;
+            const int row = nt * 8 + (lane & 7);
+            ldsm_x2(smem_u32(kv_s + row * L::kKV + ((lane >> 3) & 1) * 16 + k * 32), b0, b1);
+            mma16816(sacc[NACC == 2 ? (k & 1) : 0][n], a0, a1, a2, a3, b0, b1);
+          }
+        }
+      }
+      if (NACC == 2) {
+#pragma unroll
+        for (int n = 0; n < NTS_W; ++n)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) sacc[0][n][i] += sacc[1][n][i];
+      }
+      const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+      for (int n = 0; n < NTS_W; ++n) {
+        const int nt = wj + n * WPM;
+        if (nt < NTS) {
+          const int c = nt * 8 + 2 * t;
+          s_s[(mt * 16 + g) * L::kS + c] = sacc[0][n][0];
+          s_s[(mt * 16 + g) * L::kS + c + 1] = sacc[0][n][1];
+          s_s[(mt * 16 + g + 8) * L::kS + c] = sacc[0][n][2];
+          s_s[(mt * 16 + g + 8) * L::kS + c + 1] = sacc[0][n][3];
+        }
       }
     }
-    const int g = lane >> 2, t = lane & 3;
-#pragma unroll
-    for (int n = 0; n < NT_S; ++n) {
-      const int c = (nt0 + n) * 8 + 2 * t;
-      s_s[(mt * 16 + g) * L::kS + c] = acc[n][0];
-      s_s[(mt * 16 + g) * L::kS + c + 1] = acc[n][1];
-      s_s[(mt * 16 + g + 8) * L::kS + c] = acc[n][2];
-      s_s[(mt * 16 + g + 8) * L::kS + c + 1] = acc[n][3];
-    }
-  }
-  __syncthreads();
-  // ---- per-head softmax over this chunk (4 threads per head, 16 rows each)
-  {
-    const int h = tid >> 2, part = tid & 3;
-    if (h < HG) {
-      float v[16];
+    __syncthreads();
+    // ---- online softmax: TPH threads per head, RPT rows each
+    {
+      const int h = tid / TPH, part = tid % TPH;
+      float v[RPT];
       float mx = -INFINITY;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const int r = part * 16 + i;
-        v[i] = (r < nrows && pos_s[r] >= 0) ? s_s[h * L::kS + r] * a.scale_log2 : -INFINITY;
+      for (int i = 0; i < RPT; ++i) {
+        const int r = part * RPT + i;
+        v[i] = pos_s[r] >= 0 ? s_s[h * L::kS + r] * a.scale_log2 : -INFINITY;
         mx = fmaxf(mx, v[i]);
       }
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+#pragma unroll
+      for (int o = 1; o < TPH; o <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      const float m_old = ml_s[h * 4 + 0], l_old = ml_s[h * 4 + 1];
+      const float m_new = fmaxf(m_old, mx);
+      const float alpha = m_old == -INFINITY ? 0.f : exp2f(m_old - m_new);
       float sum = 0.f;
       uint16_t* prow = reinterpret_cast<uint16_t*>(p_s + h * L::kP);
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float p = (v[i] == -INFINITY) ? 0.f : exp2f(v[i] - mx);
-        const __nv_bfloat16 pb = __float2bfloat16_rn(p);
+      for (int i = 0; i < RPT; ++i) {
+        const float pr = v[i] == -INFINITY ? 0.f : exp2f(v[i] - m_new);
+        const __nv_bfloat16 pb = __float2bfloat16_rn(pr);
         sum += __bfloat162float(pb);      // the denominator uses exactly the weights applied to V
-        prow[part * 16 + i] = __bfloat16_as_ushort(pb);
+        prow[part * RPT + i] = __bfloat16_as_ushort(pb);
       }
-      sum += __shfl_xor_sync(0xffffffffu, sum, 1);
-      sum += __shfl_xor_sync(0xffffffffu, sum, 2);
+#pragma unroll
+      for (int o = 1; o < TPH; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (part == 0) {
-        ml_s[h * 2] = mx;
-        ml_s[h * 2 + 1] = sum;
+        ml_s[h * 4 + 0] = m_new;
+        ml_s[h * 4 + 1] = alpha * l_old + sum;
+        ml_s[h * 4 + 2] = alpha;
       }
     }
+    __syncthreads();
+    // ---- O[h][d] = alpha[h] O[h][d] + sum_r P[h][r] KV[r][d]
+    {
+      const int d0 = wj * DW, g = lane >> 2;
+      const float al0 = ml_s[(mt * 16 + g) * 4 + 2], al1 = ml_s[(mt * 16 + g + 8) * 4 + 2];
+#pragma unroll
+      for (int n = 0; n < NT_O; ++n) {
+        acc[n][0] *= al0;
+        acc[n][1] *= al0;
+        acc[n][2] *= al1;
+        acc[n][3] *= al1;
+      }
+      const uint32_t pa = smem_u32(p_s + (mt * 16 + (lane & 15)) * L::kP + (lane >> 4) * 16);
+#pragma unroll
+      for (int k = 0; k < kTile / 16; ++k) {
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(pa + k * 32, a0, a1, a2, a3);
+        const int vrow = k * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int n = 0; n < NT_O; n += 2) {
+          uint32_t b0, b1, b2, b3;
+          const int col = d0 + n * 8 + (lane >> 4) * 8;
+          ldsm_x4_t(smem_u32(kv_s + vrow * L::kKV + col * 2), b0, b1, b2, b3);
+          mma16816(acc[n], a0, a1, a2, a3, b0, b1);
+          mma16816(acc[n + 1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+    }
+    // the next tile's position pass ends with a barrier before the K/V tile is rewritten
   }
-  __syncthreads();
-  // ---- O[h][d] = sum_r P[h][r] KV[r][d]
+
+  // ---- this CTA's partial (max, sum, O) to L2, then the merge of the group
   {
-    const int mt = warp / WPM, d0 = (warp % WPM) * DW;
-    float acc[NT_O][4];
-#pragma unroll
-    for (int n = 0; n < NT_O; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-    const uint32_t pa = smem_u32(p_s + (mt * 16 + (lane & 15)) * L::kP + (lane >> 4) * 16);
-#pragma unroll
-    for (int k = 0; k < kRows / 16; ++k) {
-      uint32_t a0, a1, a2, a3;
-      ldsm_x4(pa + k * 32, a0, a1, a2, a3);
-      const int vrow = k * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-#pragma unroll
-      for (int n = 0; n < NT_O; n += 2) {
-        uint32_t b0, b1, b2, b3;
-        const int col = d0 + n * 8 + (lane >> 4) * 8;
-        ldsm_x4_t(smem_u32(kv_s + vrow * L::kKV + col * 2), b0, b1, b2, b3);
-        mma16816(acc[n], a0, a1, a2, a3, b0, b1);
-        mma16816(acc[n + 1], a0, a1, a2, a3, b2, b3);
-      }
-    }
-    const int g = lane >> 2, t = lane & 3;
+    float* po = a.part_o + ((size_t)gidx * kCl + rank) * HG * D;
+    const int d0 = wj * DW, g = lane >> 2, t = lane & 3;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-      const int h = mt * 16 + g + half * 8;
-      if (h0 + h < a.Hq) {
-        float* dst = J.part_o + (pidx + (size_t)(h0 + h) * a.n_chunks) * D;
+      float* row = po + (size_t)(mt * 16 + g + half * 8) * D + d0 + 2 * t;
 #pragma unroll
-        for (int n = 0; n < NT_O; ++n)
-          *reinterpret_cast<float2*>(dst + d0 + n * 8 + 2 * t) = make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
-      }
+      for (int n = 0; n < NT_O; ++n)
+        *reinterpret_cast<float2*>(row + n * 8) = make_float2(acc[n][2 * half], acc[n][2 * half + 1]);
     }
+    if (tid < HG) a.part_ml[((size_t)gidx * kCl + rank) * HG + tid] = make_float2(ml_s[tid * 4], ml_s[tid * 4 + 1]);
   }
-  for (int h = tid; h < HG; h += blockDim.x) {
-    if (h0 + h < a.Hq) {
-      float* ml = J.part_ml + (pidx + (size_t)(h0 + h) * a.n_chunks) * 2;
-      ml[0] = ml_s[h * 2];
-      ml[1] = ml_s[h * 2 + 1];
-    }
-  }
+  if (!a.fused) return;
+  sel_grid_sync(a.bar + gidx, kCl, a.status);
+  merge_slice<D, HG, NTHR>(a, J, q, h0, gidx, rank, s_s);
 }
 
-// Merges the chunk partials of one (job, query, head): o = sum_c 2^(m_c-M) O_c / L.
-// Each thread owns 4 output columns; every chunk's (max, sum) and partial
-// columns are loaded up front so the loads overlap.
-template <int D>
-__global__ void __launch_bounds__(D / 4) attn_combine_kernel(const __grid_constant__ AttnArgs a) {
-  constexpr int kMaxChunks = 24;
-  const int h = blockIdx.x;
-  const int job_i = blockIdx.y / a.nq, q = blockIdx.y % a.nq;
-  const AttnJob& J = a.jobs[job_i];
-  const size_t base = ((size_t)q * a.Hq + h) * a.n_chunks;
-  const int d = threadIdx.x * 4;
-  float M = -INFINITY;
-  float Lsum = 0.f;
-  float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (a.n_chunks > kMaxChunks) {   // long selections: plain two-pass loop
-    for (int c = 0; c < a.n_chunks; ++c) M = fmaxf(M, J.part_ml[(base + c) * 2]);
-    for (int c = 0; c < a.n_chunks; ++c) {
-      const float mc = J.part_ml[(base + c) * 2];
-      if (mc == -INFINITY) continue;
-      const float e = exp2f(mc - M);
-      Lsum += e * J.part_ml[(base + c) * 2 + 1];
-      const float4 vc = *reinterpret_cast<const float4*>(J.part_o + (base + c) * D + d);
-      o.x += e * vc.x;
-      o.y += e * vc.y;
-      o.z += e * vc.z;
-      o.w += e * vc.w;
-    }
-  } else {
-  float m[kMaxChunks], l[kMaxChunks];
-  float4 v[kMaxChunks];
-#pragma unroll
-  for (int c = 0; c < kMaxChunks; ++c) {
-    if (c < a.n_chunks) {
-      const float2 ml = *reinterpret_cast<const float2*>(J.part_ml + (base + c) * 2);
-      m[c] = ml.x;
-      l[c] = ml.y;
-      v[c] = ml.x == -INFINITY ? make_float4(0.f, 0.f, 0.f, 0.f)
-                               : *reinterpret_cast<const float4*>(J.part_o + (base + c) * D + d);
-      M = fmaxf(M, ml.x);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < kMaxChunks; ++c) {
-    if (c < a.n_chunks && m[c] != -INFINITY) {
-      const float e = exp2f(m[c] - M);
-      Lsum += e * l[c];
-      o.x += e * v[c].x;
-      o.y += e * v[c].y;
-      o.z += e * v[c].z;
-      o.w += e * v[c].w;
-    }
-  }
-  }
-  const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-  uint16_t* dst = J.out + ((size_t)q * a.Hq + h) * D + d;
-  const __nv_bfloat16 b[4] = {__float2bfloat16_rn(o.x * inv), __float2bfloat16_rn(o.y * inv),
-                              __float2bfloat16_rn(o.z * inv), __float2bfloat16_rn(o.w * inv)};
-  uint2 pk;
-  pk.x = (uint32_t)__bfloat16_as_ushort(b[0]) | ((uint32_t)__bfloat16_as_ushort(b[1]) << 16);
-  pk.y = (uint32_t)__bfloat16_as_ushort(b[2]) | ((uint32_t)__bfloat16_as_ushort(b[3]) << 16);
-  *reinterpret_cast<uint2*>(dst) = pk;
-  if (threadIdx.x == 0 && J.lse) J.lse[(size_t)q * a.Hq + h] = (M + log2f(Lsum)) * 0.69314718055994531f;
+// The merge of every group, when the attention CTAs could not all be resident.
+template <int D, int HG, int NTHR>
+__global__ void __launch_bounds__(NTHR) attn_merge_kernel(const __grid_constant__ AttnArgs a) {
+  using L = AttnSmem<D, HG>;
+  __shared__ float tab[(3 * kCl + 2) * HG];
+  static_assert((3 * kCl + 2) * HG * 4 <= L::kS * HG * 4, "the same tables as the fused merge");
+  const int gidx = blockIdx.z * gridDim.y + blockIdx.y;
+  const int job_i = blockIdx.z / a.nq, q = blockIdx.z % a.nq;
+  merge_slice<D, HG, NTHR>(a, a.jobs[job_i], q, blockIdx.y * HG, gidx, blockIdx.x, tab);
 }
 
-template <int D, int HG>
-cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st) {
+template <int D, int HG, int NTHR>
+cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
   using L = AttnSmem<D, HG>;
   static unsigned long long done = 0;
-  cudaError_t e = ensure_smem(sparse_attn_kernel<D, HG>, (int)L::total, done);
+  static int max_ctas[64];
+  cudaError_t e = ensure_smem(sparse_attn_kernel<D, HG, NTHR>, (int)L::total, done);
   if (e != cudaSuccess) return e;
-  const dim3 grid(a.n_chunks, (a.Hq + HG - 1) / HG, a.nq * a.n_jobs);
-  sparse_attn_kernel<D, HG><<<grid, 256, L::total, st>>>(a);
-  attn_combine_kernel<D><<<dim3(a.Hq, a.nq * a.n_jobs), D / 4, 0, st>>>(a);
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 64 && !max_ctas[dev]) {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_attn_kernel<D, HG, NTHR>, NTHR, L::total);
+    if (e != cudaSuccess) return e;
+    max_ctas[dev] = per_sm * sm_count();
+  }
+  const dim3 grid(kCl, (a.Hq + HG - 1) / HG, a.nq * a.n_jobs);
+  const int64_t ctas = (int64_t)grid.x * grid.y * grid.z;
+  a.fused = dev < 64 && ctas <= max_ctas[dev];
+  if (a.fused) {
+    e = cudaMemsetAsync(a.bar, 0, (size_t)grid.y * grid.z * sizeof(uint32_t), st);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(NTHR, 1, 1);
+    cfg.dynamicSmemBytes = L::total;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, sparse_attn_kernel<D, HG, NTHR>, a);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  sparse_attn_kernel<D, HG, NTHR><<<grid, NTHR, L::total, st>>>(a);
+  attn_merge_kernel<D, HG, NTHR><<<grid, NTHR, 0, st>>>(a);
   return cudaGetLastError();
 }
 
 }  // namespace
 
+constexpr int kAttnHG = 32;   // heads per group (fewer when Hq is smaller)
+
 size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window) {
-  const int64_t n_chunks = ((int64_t)K + window + kRows - 1) / kRows;
-  return (size_t)nq * Hq * n_chunks * ((size_t)D * 4 + 8) + 1024;
+  (void)K, (void)window;
+  const int HG = Hq <= 16 ? 16 : kAttnHG;
+  const size_t groups = (size_t)nq * ((Hq + HG - 1) / HG);
+  // partial O and (max, sum) of every CTA, barrier counts; 256-byte aligned pieces
+  return groups * kCl * HG * ((size_t)D * 4 + 8) + groups * 4 + 3 * 256;
 }
 
 // Runs n_jobs attention problems that share shapes, positions and sizes.
@@ -456,7 +529,6 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
                                     cudaStream_t st) {
   if (n_jobs < 1 || n_jobs > kMaxJobs) return cudaErrorInvalidValue;
   AttnArgs a;
-  a.n_chunks = (int32_t)(((int64_t)K + window + kRows - 1) / kRows);
   a.seq_of_query = seq_of_query;
   a.query_pos = query_pos;
   a.nq = nq;
@@ -466,7 +538,6 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
   a.n_jobs = n_jobs;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = status;
-  Carver c(ws);
   for (int j = 0; j < n_jobs; ++j) {
     AttnJob& J = a.jobs[j];
     J.q = jobs[j].q;
@@ -480,18 +551,15 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
     J.sel_cnt = jobs[j].sel_cnt;
     J.out = jobs[j].out;
     J.lse = jobs[j].lse;
-    J.part_o = c.take<float>((size_t)nq * Hq * a.n_chunks * D);
-    J.part_ml = c.take<float>((size_t)nq * Hq * a.n_chunks * 2);
   }
-  const int HG = Hq <= 16 ? 16 : (Hq <= 32 ? 32 : 64);
-  if (D == 512) {
-    if (HG == 16) return launch_attn_t<512, 16>(a, st);
-    if (HG == 32) return launch_attn_t<512, 32>(a, st);
-    return launch_attn_t<512, 64>(a, st);
-  }
-  if (HG == 16) return launch_attn_t<128, 16>(a, st);
-  if (HG == 32) return launch_attn_t<128, 32>(a, st);
-  return launch_attn_t<128, 64>(a, st);
+  const int HG = Hq <= 16 ? 16 : kAttnHG;
+  const size_t groups = (size_t)n_jobs * nq * ((Hq + HG - 1) / HG);
+  Carver c(ws);
+  a.part_o = c.take<float>(groups * kCl * HG * D);
+  a.part_ml = c.take<float2>(groups * kCl * HG);
+  a.bar = c.take<uint32_t>(groups);
+  if (D == 512) return HG == 16 ? launch_attn_t<512, 16, 256>(a, st) : launch_attn_t<512, kAttnHG, 256>(a, st);
+  return HG == 16 ? launch_attn_t<128, 16, 256>(a, st) : launch_attn_t<128, kAttnHG, 256>(a, st);
 }
 
 cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,

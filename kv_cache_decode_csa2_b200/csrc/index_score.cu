@@ -4,7 +4,7 @@
 // every query ("the first full-mode indexing layer searches the large
 // context": "DeepSeek V4.1-Flash: 552B runs like 16B", Act 2).
 //
-// Design (one persistent CTA per SM, 6 warps):
+// Design (one persistent CTA per SM, 10 warps):
 //   warp 0     TMA producer: streams 128-row key tiles (two 64-row boxes, so
 //              64-row pages work unchanged) into an NST-deep ring with evict-
 //              first L2 hints.  The key rows are the only O(context) bytes of
@@ -12,12 +12,12 @@
 //   warp 1     tcgen05 issuer: D[128 keys x N heads] = keys (K-major, swizzled)
 //              x q^T, int8 x int8 -> int32 in TMEM, double-buffered so the
 //              epilogue of tile i overlaps the MMA of tile i+1.
-//   warps 2-5  epilogue: each thread owns one key row (one TMEM lane), loads
-//              its N int32 head dots, applies ReLU and the integer head
-//              weights in registers, stores the int32 score (coalesced) and
-//              adds the score's bucket to a shared-memory radix histogram that
-//              is flushed once per query segment (the first pass of the
-//              top-k).
+//   warps 2-9  epilogue, two groups of four warps on alternate tiles: each
+//              thread owns one key row (one TMEM lane), loads its N int32
+//              head dots, applies ReLU and the integer head weights in
+//              registers, stores the int32 score (coalesced) and adds the
+//              score's bucket to a shared-memory radix histogram that is
+//              flushed once per query segment (the first pass of the top-k).
 // Work is the flat list of (query, 128-row tile) items over all queries,
 // split evenly between CTAs, so ragged batches stay balanced.
 #include "csa2_device.cuh"
@@ -48,7 +48,7 @@ struct IndexCfg {
   static constexpr int kStages = (D == 128) ? 8 : 12;         // >= 96 KiB in flight per SM
 };
 
-constexpr int kEpiThreads = 256;   // 8 epilogue warps: two per TMEM lane quarter, one per half of the heads
+constexpr int kEpiThreads = 256;   // 8 epilogue warps: two groups, one warp per TMEM lane quarter each
 __device__ __forceinline__ void named_sync_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
@@ -76,8 +76,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   uint8_t* bmat = stages + NST * TILE;
   uint32_t* hist_s = reinterpret_cast<uint32_t*>(bmat + N * D);
   int32_t* w_s = reinterpret_cast<int32_t*>(hist_s + kBuckets);
-  int32_t* part_s = w_s + 128;                                   // [2][128] partial sums of heads N/2..N-1
-  int32_t* prefix = part_s + 256;                                // [nq + 1]
+  int32_t* prefix = w_s + 128;                                   // [nq + 1]
   uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + ((a.nq + 2) & ~1));
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
@@ -112,7 +111,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     }
     for (int i = 0; i < NBUF; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kEpiThreads / 32);   // one arrival per epilogue warp
+      mbar_init(&tempty[i], kEpiThreads / 64);   // one arrival per warp of the group that reads it
     }
     mbar_init(bready, kEpiThreads / 32);
     *bound_acc = 0ull;
@@ -162,11 +161,9 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   // query) and the histogram can be swapped without any hand-off protocol.
   // `git` numbers the items of the CTA and drives every barrier phase.
   const int et = tid - 64;                 // epilogue thread 0..255 (negative for warps 0-1)
-  const int half = et >> 7;                // which half of the heads this epilogue warp sums
+  const int group = et >> 7;               // epilogue group: tiles i with i % 2 == group
   const int quarter = warp & 3;            // TMEM lanes this warp may access
   const int row = quarter * 32 + lane;     // key row of the tile this thread owns
-  constexpr int NH = N >= 64 ? N / 2 : N;  // heads per half (N <= 32: the first half takes all)
-  const bool active = N >= 64 || half == 0;
   int64_t git = 0;
   int seg_count = 0;   // segments done by this CTA (bready phase)
   int q = q0;
@@ -276,84 +273,50 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       }
     } else {
       // ---------------------------------------------------------- epilogue
-      // Two warps share each TMEM lane quarter: warps 2-5 sum heads [0, NH)
-      // and warps 6-9 heads [NH, N) of the same 128 key rows; the second
-      // group hands its partial sums over through a double-buffered shared
-      // array.  The TMEM load of tile i+1 is issued before the arithmetic of
-      // tile i, so its latency is hidden.  Every epilogue thread walks the same
-      // tiles and reaches the same named barriers even after a timeout (it
+      // Two groups of four warps (one warp per TMEM lane quarter each) take
+      // alternate tiles, so the groups never wait for each other within a
+      // segment.  A thread owns one key row: it loads the row's N head dots,
+      // frees the TMEM buffer, applies ReLU and the head weights (kept in
+      // registers) in independent partial sums, stores the score and adds
+      // its bucket to the shared histogram.  Every epilogue thread walks the
+      // same tiles and reaches the same barriers even after a timeout (it
       // then skips the TMEM reads and the stores).
-      constexpr bool kRegW = NH <= 32;       // 64 heads per half: weights stay in shared memory
-      int32_t wreg[kRegW ? NH : 1];
+      constexpr bool kRegW = N <= 64;
+      int32_t wreg[kRegW ? N : 1];
       if constexpr (kRegW) {
 #pragma unroll
-        for (int h = 0; h < NH; ++h) wreg[h] = active ? w_s[half * NH + h] : 0;
+        for (int h = 0; h < N; ++h) wreg[h] = w_s[h];
       }
-      const int32_t* wsh = w_s + half * NH;
-      auto taddr_of = [&](int64_t g) {
-        return tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((g % NBUF) * N + (active ? half * NH : 0));
-      };
-      auto wait_tile = [&](int64_t g) {
-        return __all_sync(0xffffffffu, mbar_wait(&tfull[g % NBUF], (uint32_t)((g / NBUF) & 1), abort_flag));
-      };
-      auto load = [&](uint32_t (&r)[NH], int64_t g) {
-        if constexpr (NH == 16) {
-          tmem_ld16(taddr_of(g), r);
-        } else {
-#pragma unroll
-          for (int c = 0; c < NH / 32; ++c)
-            tmem_ld32(taddr_of(g) + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
-        }
-      };
-      // one tile: `cur` holds its accumulators; prefetch the next tile into `nxt`
-      auto step = [&](uint32_t (&cur)[NH], bool okc, uint32_t (&nxt)[NH], bool& okn, int i) {
+      for (int i = group; i < n_it; i += 2) {
         const int64_t g = git + i;
-        const bool has_next = i + 1 < n_it;
-        if (has_next) {
-          okn = wait_tile(g + 1);
-          if (okn) {
-            tc_fence_after();
-            load(nxt, g + 1);
-          }
-        }
-        int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent chains, no long serial sum
-#pragma unroll
-        for (int h = 0; h < NH; ++h) part[h & 7] += (kRegW ? wreg[h] : wsh[h]) * max((int32_t)cur[h], 0);
-        int32_t s = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-        if (!active) s = 0;
-        if (half == 1) part_s[(g & 1) * 128 + row] = s;
-        named_sync_epi();
-        if (half == 0 && okc) {
-          s += part_s[(g & 1) * 128 + row];
-          const int32_t pos = (tile0 + i) * 128 + row;
-          if (pos <= pos_q) {
-            a.scores[(int64_t)q * a.ld + pos] = s;
-            atomicAdd(&hist_s[score_bucket(s)], 1u);
-          }
-        }
-        if (has_next) {
-          if (okn) tmem_wait_ld();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&tempty[(g + 1) % NBUF]);
-        }
-      };
-      uint32_t ra[NH], rb[NH];
-      bool oka = false, okb = false;
-      if (n_it > 0) {
-        oka = wait_tile(git);
-        if (oka) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[g % NBUF], (uint32_t)((g / NBUF) & 1), abort_flag));
+        uint32_t r[N];
+        if (ok) {
           tc_fence_after();
-          load(ra, git);
+          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((g % NBUF) * N);
+          if constexpr (N == 16) {
+            tmem_ld16(taddr, r);
+          } else {
+#pragma unroll
+            for (int c = 0; c < N / 32; ++c)
+              tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+          }
           tmem_wait_ld();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[git % NBUF]);
-      }
-      for (int i = 0; i < n_it; i += 2) {
-        step(ra, oka, rb, okb, i);
-        if (i + 1 < n_it) step(rb, okb, ra, oka, i + 1);
+        if (lane == 0) mbar_arrive(&tempty[g % NBUF]);
+        if (ok) {
+          int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent chains, no long serial sum
+#pragma unroll
+          for (int h = 0; h < N; ++h) part[h & 7] += (kRegW ? wreg[h] : w_s[h]) * max((int32_t)r[h], 0);
+          const int32_t sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+          const int32_t pos = (tile0 + i) * 128 + row;
+          if (pos <= pos_q) {
+            a.scores[(int64_t)q * a.ld + pos] = sc;
+            atomicAdd(&hist_s[score_bucket(sc)], 1u);
+          }
+        }
       }
       // this query's histogram goes to global memory
       named_sync_epi();
@@ -404,7 +367,7 @@ EncodeTiledFn encode_fn() {
 template <int D>
 size_t index_smem_bytes(int N, int nq) {
   using Cfg = IndexCfg<D>;
-  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)N * D + kBuckets * 4 + 128 * 4 + 256 * 4 +
+  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)N * D + kBuckets * 4 + 128 * 4 +
          (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 + 32;
 }
 

@@ -44,25 +44,27 @@ __device__ __forceinline__ uint64_t sel_scan(uint64_t v, uint64_t* wtmp, uint64_
 }
 
 // Barrier of the G co-resident CTAs of one row: waits until `bar` (zeroed
-// before the launch) reaches `target`, a multiple of G.  Bounded: after
-// kWaitLimitNs it records CSA2_ERR_TIMEOUT and goes on.
+// before the launch) reaches `target`, a multiple of G.  The block barrier
+// orders the CTA's writes before thread 0's release-add; thread 0's acquire
+// load, then the block barrier, order the other CTAs' writes before every
+// later read.  Bounded: after kWaitLimitNs it records CSA2_ERR_TIMEOUT and
+// goes on.
 __device__ __forceinline__ void sel_grid_sync(uint32_t* bar, uint32_t target, int32_t* status) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(bar, 1u);
-    const uint64_t t0 = global_ns();
-    while (true) {
-      uint32_t v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
-      if (v >= target) break;
-      if (global_ns() - t0 > kWaitLimitNs) {
-        record_error(status, CSA2_ERR_TIMEOUT);
-        break;
-      }
-      __nanosleep(32);
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+    if (v < target) {
+      const uint64_t t0 = global_ns();
+      do {
+        if (global_ns() - t0 > kWaitLimitNs) {
+          record_error(status, CSA2_ERR_TIMEOUT);
+          break;
+        }
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(bar) : "memory");
+      } while (v < target);
     }
-    __threadfence();
   }
   __syncthreads();
 }

@@ -132,7 +132,7 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   int32_t* sc = scores ? scores : sc_ws;
   const int64_t ld = scores ? ld_scores : max_ctx;
   const bool topk = P > 0 || K > 0;
-  if (topk) {
+  if (topk && !launch_opts().prezeroed) {
     cudaError_t e = cudaMemsetAsync(ts.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
   }
@@ -333,6 +333,34 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
       sel_cnt_of[i] = ly.sel_cnt ? ly.sel_cnt : p.sel_cnt[i];
     }
   }
+  // One launch zeroes all scratch of the step up front when every piece is
+  // used once (one FULL layer, at most one reindex launch), so the kernels of
+  // the step then follow one another as programmatic dependents.
+  int n_full = 0, n_reindex = 0;
+  for (int i = 0; i < L; ++i) {
+    n_full += modes[i] == CSA2_FULL;
+    n_reindex += modes[i] == CSA2_REINDEX;
+  }
+  LaunchOpts opts;
+  if (n_full == 1 && n_reindex <= kMaxReindexJobs) {
+    void* zp[3];
+    size_t zb[3];
+    int nz = 0;
+    TopkScratch ts;
+    index_full_ws(s->nq, s->max_ctx, s->P, s->K, p.index_base, nullptr, &ts);
+    zp[nz] = ts.hist;
+    zb[nz++] = topk_zero_bytes(s->nq);
+    if (n_reindex > 0) {
+      zp[nz] = p.reindex_base;   // the fused launch's histograms and headers lead its scratch
+      zb[nz++] = (size_t)n_reindex * s->nq * (kBuckets + 4) * sizeof(uint32_t);
+    }
+    attn_bar_region(p.attn_base, L, s->nq, s->Hq, s->D, &zp[nz], &zb[nz]);
+    ++nz;
+    if (launch_zero(zp, zb, nz, st) != cudaSuccess) return CSA2_ERR_CUDA;
+    opts.pdl = true;
+    opts.prezeroed = true;
+  }
+  LaunchOptsScope scope(opts);
   // Every FULL layer, then in one launch the REINDEX layers that search its pool.
   for (int i = 0; i < L; ++i) {
     if (modes[i] != CSA2_FULL) continue;

@@ -31,6 +31,14 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// Programmatic dependent launch.  pdl_wait() blocks until the grid this one
+// depends on has completed and its writes are visible (a no-op when the
+// launch has no such dependency); pdl_trigger() lets the next grid of the
+// stream be launched early.  Work before pdl_wait() may touch only inputs that
+// no earlier grid of the stream writes.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred = 0;
   asm volatile(

@@ -141,6 +141,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_trigger();   // the next grid may be launched (it waits for this one to finish)
 
   const int64_t total = prefix[a.nq];
   const int64_t lo = total * blockIdx.x / gridDim.x;
@@ -281,6 +282,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       // its bucket to the shared histogram.  Every epilogue thread walks the
       // same tiles and reaches the same barriers even after a timeout (it
       // then skips the TMEM reads and the stores).
+      if (seg_count == 0) pdl_wait();   // scores and histogram: after the grid before (it zeroes them)
       constexpr bool kRegW = N <= 64;
       int32_t wreg[kRegW ? N : 1];
       if constexpr (kRegW) {
@@ -377,8 +379,8 @@ cudaError_t launch_one(const CUtensorMap& map, const IndexArgs& a, int grid, cud
   static unsigned long long done = 0;
   cudaError_t e = ensure_smem(index_score_kernel<D, N>, (int)index_smem_bytes<D>(N, kMaxQueries), done);
   if (e != cudaSuccess) return e;
-  index_score_kernel<D, N><<<grid, 64 + kEpiThreads, smem, st>>>(map, a);
-  return cudaGetLastError();
+  return launch_k(index_score_kernel<D, N>, dim3(grid), dim3(64 + kEpiThreads), smem, st, false, launch_opts().pdl,
+                  map, a);
 }
 
 }  // namespace

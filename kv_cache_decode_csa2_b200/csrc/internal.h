@@ -23,6 +23,36 @@ struct Carver {
   }
 };
 
+// Options for the launches inside one layer-plan call (per host thread):
+//   pdl        launch the index-score, select, reindex and attention kernels
+//              as programmatic dependents of the kernel before them;
+//   prezeroed  the top-k, reindex and attention scratch was zeroed by the
+//              caller (in the kernel launched just before).
+struct LaunchOpts {
+  bool pdl = false;
+  bool prezeroed = false;
+};
+LaunchOpts& launch_opts();
+struct LaunchOptsScope {   // sets the options for its lifetime
+  LaunchOpts saved;
+  explicit LaunchOptsScope(LaunchOpts o) : saved(launch_opts()) { launch_opts() = o; }
+  ~LaunchOptsScope() { launch_opts() = saved; }
+};
+// Zeroes up to kMaxZeroRegions regions (4-byte multiples) in one launch.
+constexpr int kMaxZeroRegions = 4;
+cudaError_t launch_zero(void* const* ptrs, const size_t* bytes, int n, cudaStream_t st);
+// Launches `kernel` with the cooperative and programmatic-dependence
+// attributes asked for.  A programmatic launch the device refuses is retried
+// once without the attribute, and programmatic launches stay off from then on.
+cudaError_t launch_ex(const void* kernel, void** args, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                      bool cooperative, bool pdl);
+template <class... Args>
+cudaError_t launch_k(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     bool cooperative, bool pdl, Args... args) {
+  void* argv[] = {static_cast<void*>(&args)...};
+  return launch_ex(reinterpret_cast<const void*>(kernel), argv, grid, block, smem, st, cooperative, pdl);
+}
+
 // Radix top-k scratch for nq queries and up to two thresholds per query.
 struct TopkScratch {
   uint32_t* hist;        // [nq][kBuckets]                 (zeroed before the histogram pass)
@@ -172,6 +202,7 @@ struct AttnJobDesc {
   float* lse;
 };
 constexpr int kMaxAttnJobs = 16;
+void attn_bar_region(void* ws, int32_t n_jobs, int32_t nq, int32_t Hq, int32_t D, void** ptr, size_t* bytes);
 cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const int32_t* seq_of_query,
                                     const int32_t* query_pos, int32_t nq, int32_t Hq, int32_t D,
                                     int32_t K, int32_t window, float scale, void* ws, int32_t* status,

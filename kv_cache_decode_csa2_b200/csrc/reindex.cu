@@ -226,6 +226,36 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   const RSelJob& J = a.job[jb];
   const int prob = jb * a.nq + q;
   const int G = a.G;
+  if (tid == 0) {
+    bstar_s = -1;
+    above_s = 0;
+    own_cnt = 0;
+    kthr_s = ~0ull;
+  }
+
+  // ---- prologue on this layer's own inputs: TMEM, the MMA barrier, the
+  // query rows (B operand) and the head weights
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    fence_mbar_init();
+  }
+  {
+    const int8_t* qsrc = J.q + (int64_t)q * a.H * D;
+    for (int idx = tid; idx < N * (D / 16); idx += NT) {
+      const int r = idx / (D / 16), c = idx % (D / 16);
+      int4 v = make_int4(0, 0, 0, 0);
+      if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
+      *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
+    }
+    if (tid < N) w_s[tid] = tid < a.H ? (int32_t)__ldg(J.w + (int64_t)q * a.H + tid) : 0;
+  }
+  pdl_wait();      // the pool comes from the grid before
+  pdl_trigger();
+
   int32_t cnt = __ldg(a.pool_cnt + q);
   cnt = cnt < 0 ? 0 : (cnt > a.P ? a.P : cnt);
   const int32_t slot0 = x * NT, slot = slot0 + tid;
@@ -234,26 +264,12 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   const int32_t* pidx = a.pool_idx + (int64_t)q * a.P;
   const int32_t pos = valid ? __ldg(pidx + slot) : -1;
   const int32_t prev = (valid && slot > 0) ? __ldg(pidx + slot - 1) : INT32_MIN;
-  if (tid == 0) {
-    bstar_s = -1;
-    above_s = 0;
-    own_cnt = 0;
-    kthr_s = ~0ull;
-  }
   if (valid && pos <= prev) record_error(a.status, CSA2_ERR_ORDER);   // pool positions ascend
 
   // ---- scores of this CTA's NT pool entries (one per thread)
   int32_t s = 0;
   if (has) {
     const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
-    if (warp == 0) {
-      tmem_alloc(tmem_slot, TMEM_COLS);
-      tmem_relinquish();
-    }
-    if (tid == 0) {
-      mbar_init(bar, 1);
-      fence_mbar_init();
-    }
     {
       const uint8_t* src = nullptr;
       if (valid) {
@@ -269,20 +285,14 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
         else *reinterpret_cast<int4*>(dst) = make_int4(0, 0, 0, 0);
       }
     }
-    const int8_t* qsrc = J.q + (int64_t)q * a.H * D;
-    for (int idx = tid; idx < N * (D / 16); idx += NT) {
-      const int r = idx / (D / 16), c = idx % (D / 16);
-      int4 v = make_int4(0, 0, 0, 0);
-      if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
-      *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
-    }
-    if (tid < N) w_s[tid] = tid < a.H ? (int32_t)__ldg(J.w + (int64_t)q * a.H + tid) : 0;
     cp_async_wait_all();
     fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem_base = *tmem_slot;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  if (has) {
     if (tid == 0) {
       constexpr uint32_t idesc = idesc_i8(128, N);
       const uint32_t a_addr = smem_u32(atile), b_addr = smem_u32(bmat);
@@ -319,12 +329,12 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     } else if (tid == 0) {
       record_error(a.status, CSA2_ERR_TIMEOUT);
     }
-    tc_fence_before();
-    __syncthreads();   // also: the tiles are free for the tie list from here on
-    if (warp == 0) {
-      tc_fence_after();
-      tmem_dealloc(tmem_base, TMEM_COLS);
-    }
+  }
+  tc_fence_before();
+  __syncthreads();   // also: the tiles are free for the tie list from here on
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
   if (J.scores && valid) J.scores[(int64_t)q * a.P + slot] = s;
 
@@ -455,21 +465,12 @@ cudaError_t launch_rs_t(const RSelArgs& a_in, int n_jobs, int nq, size_t zero_by
   RSelArgs a = a_in;
   a.G = (a.P + Lay::NT - 1) / Lay::NT;
   if ((int64_t)a.G * nq * n_jobs > max_ctas[dev]) return cudaErrorNotSupported;
-  e = cudaMemsetAsync(a.hist, 0, zero_bytes, st);   // histograms and barrier headers
-  if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.G, nq, n_jobs);
-  cfg.blockDim = dim3(Lay::NT, 1, 1);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, reindex_select_kernel<D, N, T>, a);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  if (!launch_opts().prezeroed) {
+    e = cudaMemsetAsync(a.hist, 0, zero_bytes, st);   // histograms and barrier headers
+    if (e != cudaSuccess) return e;
+  }
+  return launch_k(reindex_select_kernel<D, N, T>, dim3(a.G, nq, n_jobs), dim3(Lay::NT), smem, st, true,
+                  launch_opts().pdl, a);
 }
 
 // Two tiles per CTA when the CTAs fit on the device, else four.

@@ -242,7 +242,6 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
                           : make_int4(0, 0, 0, 0);
   }
   const int32_t pos = __ldg(a.query_pos + q);
-  int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
   const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
 #pragma unroll
   for (int i = 0; i < QPER; ++i) {
@@ -253,6 +252,9 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
     ml_s[tid * 4 + 0] = -INFINITY;
     ml_s[tid * 4 + 1] = 0.f;
   }
+  pdl_wait();      // the selection comes from the grid before
+  pdl_trigger();
+  int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
   if (tid == 0 && rank == 0 && pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
 
   // ---- this CTA's rows: selection entries [e0, e1) below the window start,
@@ -489,21 +491,11 @@ cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
   const int64_t ctas = (int64_t)grid.x * grid.y * grid.z;
   a.fused = dev < 64 && ctas <= max_ctas[dev];
   if (a.fused) {
-    e = cudaMemsetAsync(a.bar, 0, (size_t)grid.y * grid.z * sizeof(uint32_t), st);
-    if (e != cudaSuccess) return e;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(NTHR, 1, 1);
-    cfg.dynamicSmemBytes = L::total;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, sparse_attn_kernel<D, HG, NTHR>, a);
-    if (e != cudaSuccess) return e;
-    return cudaGetLastError();
+    if (!launch_opts().prezeroed) {
+      e = cudaMemsetAsync(a.bar, 0, (size_t)grid.y * grid.z * sizeof(uint32_t), st);
+      if (e != cudaSuccess) return e;
+    }
+    return launch_k(sparse_attn_kernel<D, HG, NTHR>, grid, dim3(NTHR), L::total, st, true, launch_opts().pdl, a);
   }
   sparse_attn_kernel<D, HG, NTHR><<<grid, NTHR, L::total, st>>>(a);
   attn_merge_kernel<D, HG, NTHR><<<grid, NTHR, 0, st>>>(a);
@@ -520,6 +512,18 @@ size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t 
   const size_t groups = (size_t)nq * ((Hq + HG - 1) / HG);
   // partial O and (max, sum) of every CTA, barrier counts; 256-byte aligned pieces
   return groups * kCl * HG * ((size_t)D * 4 + 8) + groups * 4 + 3 * 256;
+}
+
+// The barrier counts inside an attention workspace of n_jobs layers: they must
+// be zero before a launch that merges in place.
+void attn_bar_region(void* ws, int32_t n_jobs, int32_t nq, int32_t Hq, int32_t D, void** ptr, size_t* bytes) {
+  const int HG = Hq <= 16 ? 16 : kAttnHG;
+  const size_t groups = (size_t)n_jobs * nq * ((Hq + HG - 1) / HG);
+  Carver c(ws);
+  c.take<float>(groups * kCl * HG * D);
+  c.take<float2>(groups * kCl * HG);
+  *ptr = c.take<uint32_t>(groups);
+  *bytes = groups * sizeof(uint32_t);
 }
 
 // Runs n_jobs attention problems that share shapes, positions and sizes.

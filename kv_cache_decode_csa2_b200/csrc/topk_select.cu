@@ -91,7 +91,6 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = blockIdx.y, c = blockIdx.x, G = a.G, n_k = a.n_k;
-  const int32_t n = sel_n(a, q);
   const int32_t j0 = c * kSpan + tid * E;
   const int32_t* row = a.scores + (int64_t)q * a.ld;
   uint32_t phase = 0;   // grid barriers passed
@@ -102,6 +101,9 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
     own_cnt[tid] = 0;
     kthr_s[tid] = ~0ull;
   }
+  pdl_wait();      // the scores, the histogram and the counts come from the grid before
+  pdl_trigger();
+  const int32_t n = sel_n(a, q);
 
   // ---- 1. loads: scores (up to n_max, which the row always holds; masked by
   // n below), this thread's histogram bins when given, the order check
@@ -388,19 +390,9 @@ cudaError_t launch_select(const int32_t* scores, int64_t ld, const int32_t* n_va
     a.out_cnt[t] = o.cnt;
   }
   a.status = status;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(G, nq, 1);
-  cfg.blockDim = dim3(kSelNT, 1, 1);
-  cfg.dynamicSmemBytes = kSelSmem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = G > 1 ? 1 : 0;
-  e = one ? cudaLaunchKernelEx(&cfg, select_kernel<16>, a) : cudaLaunchKernelEx(&cfg, select_kernel<8>, a);
-  if (e != cudaSuccess) return e;
-  return cudaGetLastError();
+  const bool pdl = launch_opts().pdl;
+  return one ? launch_k(select_kernel<16>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, G > 1, pdl, a)
+             : launch_k(select_kernel<8>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, G > 1, pdl, a);
 }
 
 }  // namespace csa2

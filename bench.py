@@ -234,12 +234,14 @@ def algorithmic_bytes(wl, layers, pos) -> tuple[int, dict]:
 
 
 def kernels_per_step(wl) -> int:
-    """Kernels one step launches: the index-score stream, the select/resolve/
-    write passes of the pool top-k, a scorer and a top-k kernel per reindex
-    layer, and the attention and combine kernels for all layers."""
+    """Kernels one plan step launches on this workload: one launch that zeroes
+    the step's scratch, the index-score stream and the pool select of the full
+    layer, one fused scoring + top-k launch for the reindex layers of the pool,
+    and one attention launch for all layers (the ncu launch list in profiles/
+    shows the same five per step)."""
     n_re = sum(1 for m in wl.modes if m == synth.REINDEX)
     n_full = sum(1 for m in wl.modes if m == synth.FULL)
-    return n_full * 4 + n_re * 2 + 2
+    return 1 + 2 * n_full + (1 if n_re else 0) + 1
 
 
 # ----------------------------------------------------------------- the CPU oracle baseline

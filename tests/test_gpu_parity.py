@@ -245,6 +245,34 @@ def test_reindex_batch_of_many_queries():
         assert np.array_equal(sels[i, :len(ref_sel)], ref_sel)
 
 
+# ------------------------------------------------------------------ A6 prefill chunk
+def test_prefill_chunk_matches_oracle():
+    """A causal prefill chunk (the C4 shape, reduced): 96 queries at positions
+    8904..8999 of one 9000-row sequence.  Every query scores its own prefix,
+    keeps its top-512 of the whole prefix (no pool) and attends to it plus the
+    window.  Sampled queries are checked against the oracle one by one."""
+    wl = synth.scaled(synth.C4_PREFILL, seq_lens=(9000,), prefill=(96, 8904))
+    c = G.build(wl)
+    ly = c.layers_dev[0]
+    nq = len(c.query_pos)
+    B.check_status(B.csa2_index_full(ly.q, ly.w, ly.keys, c.pos_dev, c.max_ctx, seq_of_query=c.seq_dev,
+                                     K=wl.topk, sel_idx=ly.sel_idx, sel_cnt=ly.sel_cnt))
+    B.check_status(B.csa2_sparse_attn_fp4(ly.q_attn, ly.codes, ly.scales, c.pos_dev, ly.sel_idx, ly.out,
+                                          sel_cnt=ly.sel_cnt, seq_of_query=c.seq_dev, window=wl.window,
+                                          lse=ly.lse))
+    sels, cnts, outs = _np(ly.sel_idx), _np(ly.sel_cnt), _np(ly.out.float())
+    keys = c.host_keys[(0, 0)]
+    codes, scales = c.fp4_host[(0, 0)]
+    for i in (0, 1, 17, 50, 94, 95):
+        q, w = c.host_q[(0, i)]
+        sel, S, o, _ = O.prefill_query(q, w, keys, c.host_qa[(0, i)], codes, scales, int(c.query_pos[i]),
+                                       wl.topk, wl.window)
+        assert cnts[i] == len(sel) and np.array_equal(sels[i, :cnts[i]], sel), f"query {i}"
+        ok, err = G.tol_ok(outs[i], o)
+        assert ok, f"query {i}: max abs err {err}"
+    assert nq == 96
+
+
 # ------------------------------------------------------------------ K4 attention
 @pytest.mark.parametrize("wl", [synth.C0_TINY, synth.scaled(synth.C1_SINGLE, seq_lens=(3001,))],
                          ids=["hq8_d128", "hq64_d512"])

@@ -136,8 +136,9 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
     cudaError_t e = cudaMemsetAsync(ts.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
   }
+  bool hist_built = false;
   cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,
-                                     topk ? ts.hist : nullptr, status, st);
+                                     topk ? ts.hist : nullptr, status, st, &hist_built);
   if (e != cudaSuccess) return CSA2_ERR_CUDA;
   if (!topk) return CSA2_OK;
   TopkOut outs[2];
@@ -145,7 +146,7 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   if (P > 0) outs[n++] = TopkOut{pool_idx, pool_cnt, P};
   if (K > 0) outs[n++] = TopkOut{sel_idx, sel_cnt, K};
   return cuda_status(launch_topk_large(sc, ld, nullptr, query_pos, nullptr, nq, max_ctx, outs, n, ts,
-                                       true, status, st));
+                                       hist_built, status, st));
 }
 
 size_t csa2_topk_pool_workspace(int32_t nq, int32_t n_max, int32_t k) {

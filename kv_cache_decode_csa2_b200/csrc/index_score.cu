@@ -41,6 +41,7 @@ struct IndexArgs {
 };
 
 constexpr int kMaxQueries = 4096;   // per launch (the work list prefix lives in shared memory)
+constexpr int kGroupMinQueries = 16;   // from this many queries on, queries of a sequence share key tiles
 
 template <int D>
 struct IndexCfg {
@@ -59,25 +60,31 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   return true;
 }
 
-template <int D, int N>
+// QG queries of one sequence share each key tile (QG = 1 for decode; 4 for a
+// prefill chunk, where consecutive queries of a sequence form the groups).
+template <int D, int N, int QG>
 __global__ void __launch_bounds__(64 + kEpiThreads, 1)
 index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) {
   using Cfg = IndexCfg<D>;
   constexpr int NST = Cfg::kStages;
   constexpr int TILE = Cfg::kTile;
+  constexpr int NG = N * QG;            // MMA N: the heads of every query of a group
+  static_assert(NG <= 256, "one MMA covers the group");
   // As many TMEM accumulator buffers as fit in the 512 columns (at most 8),
   // so the MMA can run up to NBUF tiles ahead of the epilogue.
-  constexpr int NBUF = (512 / N) < 8 ? (512 / N) : 8;
-  constexpr uint32_t TMEM_COLS = NBUF * N <= 32 ? 32 : NBUF * N <= 64 ? 64 : NBUF * N <= 128 ? 128 : NBUF * N <= 256 ? 256 : 512;
+  constexpr int NBUF = (512 / NG) < 8 ? (512 / NG) : 8;
+  constexpr uint32_t TMEM_COLS = NBUF * NG <= 32 ? 32 : NBUF * NG <= 64 ? 64 : NBUF * NG <= 128 ? 128 : NBUF * NG <= 256 ? 256 : 512;
+  constexpr int kHist = QG == 1 ? kBuckets : 0;   // grouped launches leave the histogram to the top-k
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
   uint8_t* bmat = stages + NST * TILE;
-  uint32_t* hist_s = reinterpret_cast<uint32_t*>(bmat + N * D);
-  int32_t* w_s = reinterpret_cast<int32_t*>(hist_s + kBuckets);
-  int32_t* prefix = w_s + 128;                                   // [nq + 1]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(prefix + ((a.nq + 2) & ~1));
+  uint32_t* hist_s = reinterpret_cast<uint32_t*>(bmat + NG * D);
+  int32_t* w_s = reinterpret_cast<int32_t*>(hist_s + kHist);     // [NG] (at least 128)
+  int32_t* prefix = w_s + (NG > 128 ? NG : 128);                 // [groups + 1] tiles before each group
+  int32_t* gq = prefix + ((a.nq + 2) & ~1);                      // [groups + 1] first query of each group
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gq + ((a.nq + 2) & ~1));
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
   uint64_t* tfull = bars + 2 * NST;
@@ -85,26 +92,21 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   uint64_t* bready = tempty + NBUF;                              // the segment's B operand is in place
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bready + 2);
   volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(tmem_slot + 1);
-  unsigned long long* bound_acc = reinterpret_cast<unsigned long long*>(tmem_slot + 2);
+  int32_t* ngroups_s = const_cast<int32_t*>(abort_flag) + 1;
+  unsigned long long* bound_acc = reinterpret_cast<unsigned long long*>(tmem_slot + 4);   // [QG]
+  int32_t* mpos = reinterpret_cast<int32_t*>(bound_acc + QG);                         // [QG] member positions
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- work list: prefix[q+1] = tiles of query q (0 for an invalid position)
+  // ---- groups: runs of consecutive queries of one sequence, cut every QG
   for (int i = tid; i < a.nq; i += blockDim.x) {
     const int32_t pos = __ldg(a.query_pos + i);
-    int32_t t = 0;
-    if (pos < 0 || pos >= a.max_ctx) {
-      record_error(a.status, CSA2_ERR_INDEX_RANGE);
-    } else {
-      t = (pos + 128) / 128;
-    }
-    prefix[i + 1] = t;
+    if (pos < 0 || pos >= a.max_ctx) record_error(a.status, CSA2_ERR_INDEX_RANGE);
   }
-  for (int i = tid; i < kBuckets; i += blockDim.x) hist_s[i] = 0;
+  for (int i = tid; i < kHist; i += blockDim.x) hist_s[i] = 0;
   if (tid == 0) {
-    prefix[0] = 0;
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
@@ -114,7 +116,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       mbar_init(&tempty[i], kEpiThreads / 64);   // one arrival per warp of the group that reads it
     }
     mbar_init(bready, kEpiThreads / 32);
-    *bound_acc = 0ull;
+    for (int k = 0; k < QG; ++k) bound_acc[k] = 0ull;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -122,18 +124,64 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 0) {
+    if constexpr (QG == 1) {
+      for (int i = lane; i <= a.nq; i += 32) gq[i] = i;
+      if (lane == 0) *ngroups_s = a.nq;
+    } else {
+      int32_t last_start = 0, n_groups = 0;
+      for (int base = 0; base < a.nq; base += 32) {
+        const int i = base + lane;
+        const bool valid = i < a.nq;
+        bool s = false;
+        if (valid) {
+          const int32_t sq = a.seq_of_query ? __ldg(a.seq_of_query + i) : i;
+          const int32_t sp = i == 0 ? -1 : (a.seq_of_query ? __ldg(a.seq_of_query + i - 1) : i - 1);
+          s = i == 0 || sq != sp;
+        }
+        int32_t v = s ? i : -1;   // latest run start at or before i
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v = v > n ? v : n;
+        }
+        v = v > last_start ? v : last_start;
+        const bool f = valid && (s || (i - v) % QG == 0);
+        const uint32_t bal = __ballot_sync(0xffffffffu, f);
+        if (f) gq[n_groups + __popc(bal & ((1u << lane) - 1u))] = i;
+        n_groups += __popc(bal);
+        last_start = __shfl_sync(0xffffffffu, v, 31);
+      }
+      if (lane == 0) {
+        gq[n_groups] = a.nq;
+        *ngroups_s = n_groups;
+      }
+    }
+  }
+  __syncthreads();
+  const int ngroups = *ngroups_s;
+  // prefix[g+1] = tiles of group g: the longest causal prefix of its queries
+  for (int g = tid; g < ngroups; g += blockDim.x) {
+    int32_t t = 0;
+    for (int i = gq[g]; i < gq[g + 1]; ++i) {
+      const int32_t pos = __ldg(a.query_pos + i);
+      if (pos >= 0 && pos < a.max_ctx && (pos + 128) / 128 > t) t = (pos + 128) / 128;
+    }
+    prefix[g + 1] = t;
+  }
+  if (tid == 0) prefix[0] = 0;
   __syncthreads();
   if (warp == 0) {   // inclusive scan of tile counts, 32 at a time
     int32_t carry = 0;
-    for (int base = 0; base < a.nq; base += 32) {
+    for (int base = 0; base < ngroups; base += 32) {
       const int i = base + lane;
-      int32_t v = (i < a.nq) ? prefix[i + 1] : 0;
+      int32_t v = (i < ngroups) ? prefix[i + 1] : 0;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += n;
       }
-      if (i < a.nq) prefix[i + 1] = v + carry;
+      if (i < ngroups) prefix[i + 1] = v + carry;
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
   }
@@ -143,23 +191,23 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const uint32_t tmem_base = *tmem_slot;
   pdl_trigger();   // the next grid may be launched (it waits for this one to finish)
 
-  const int64_t total = prefix[a.nq];
+  const int64_t total = prefix[ngroups];
   const int64_t lo = total * blockIdx.x / gridDim.x;
   const int64_t hi = total * (blockIdx.x + 1) / gridDim.x;
-  int q0 = 0;
+  int g0 = 0;
   {
-    int l = 0, r = a.nq - 1;   // last q with prefix[q] <= lo
+    int l = 0, r = ngroups > 0 ? ngroups - 1 : 0;   // last group with prefix[g] <= lo
     while (l < r) {
       const int m = (l + r + 1) >> 1;
       if (prefix[m] <= lo) l = m; else r = m - 1;
     }
-    q0 = l;
+    g0 = l;
   }
 
-  // The CTA's items are processed one query segment at a time.  Within a
+  // The CTA's items are processed one group segment at a time.  Within a
   // segment the producer, the MMA issuer and the epilogue run as a pipeline.
   // Between segments the whole CTA synchronises, so the B operand (the
-  // query) and the histogram can be swapped without any hand-off protocol.
+  // queries) and the histogram can be swapped without any hand-off protocol.
   // `git` numbers the items of the CTA and drives every barrier phase.
   const int et = tid - 64;                 // epilogue thread 0..255 (negative for warps 0-1)
   const int group = et >> 7;               // epilogue group: tiles i with i % 2 == group
@@ -167,45 +215,56 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int row = quarter * 32 + lane;     // key row of the tile this thread owns
   int64_t git = 0;
   int seg_count = 0;   // segments done by this CTA (bready phase)
-  int q = q0;
+  int g = g0;
   for (int64_t s_lo = lo; s_lo < hi;) {
-    while (s_lo >= prefix[q + 1]) ++q;
-    const int64_t s_hi = hi < (int64_t)prefix[q + 1] ? hi : (int64_t)prefix[q + 1];
+    while (s_lo >= prefix[g + 1]) ++g;
+    const int64_t s_hi = hi < (int64_t)prefix[g + 1] ? hi : (int64_t)prefix[g + 1];
     const int n_it = (int)(s_hi - s_lo);
-    const int32_t tile0 = (int32_t)(s_lo - prefix[q]);
-    const int32_t pos_q = __ldg(a.query_pos + q);
+    const int32_t tile0 = (int32_t)(s_lo - prefix[g]);
+    const int q0 = gq[g], nm = gq[g + 1] - gq[g];   // the group's queries
+    int32_t pos_hi = -1;                            // last position any of them sees
+    for (int k = 0; k < nm; ++k) {
+      const int32_t p = __ldg(a.query_pos + q0 + k);
+      if (p < a.max_ctx && p > pos_hi) pos_hi = p;
+    }
 
-    // ---- segment set-up (epilogue threads): B operand = q rows 0..H-1, zero
-    // rows up to N, K-major with the tile swizzle, and the head weights.  The
-    // producer does not wait for it (key tiles do not depend on the query);
-    // the MMA issuer waits on `bready`.  The int32 overflow guard
-    // 128 * sum_h |w_h| * sum_d |q_hd| < 2^31 is checked off the critical path.
-    const int8_t* qsrc = a.q + (int64_t)q * a.H * D;
+    // ---- segment set-up (epilogue threads): B operand = the group's q rows
+    // (query k at rows k N .. k N + H - 1, zero rows elsewhere), K-major with
+    // the tile swizzle, and the head weights.  The producer does not wait for
+    // it (key tiles do not depend on the queries); the MMA issuer waits on
+    // `bready`.  The int32 overflow guard 128 * sum_h |w_h| * sum_d |q_hd| <
+    // 2^31 is checked per query off the critical path.
     if (warp >= 2) {
-      for (int idx = et; idx < N * (D / 16); idx += kEpiThreads) {
+      for (int idx = et; idx < NG * (D / 16); idx += kEpiThreads) {
         const int r = idx / (D / 16), c = idx % (D / 16);
+        const int k = r / N, h = r % N;
         int4 v = make_int4(0, 0, 0, 0);
-        if (r < a.H) v = __ldg(reinterpret_cast<const int4*>(qsrc + r * D) + c);
+        if (k < nm && h < a.H) v = __ldg(reinterpret_cast<const int4*>(a.q + ((int64_t)(q0 + k) * a.H + h) * D) + c);
         *reinterpret_cast<int4*>(bmat + swizzled_chunk(r, c, D)) = v;
       }
-      if (et < N) w_s[et] = et < a.H ? (int32_t)__ldg(a.w + (int64_t)q * a.H + et) : 0;
+      for (int r = et; r < NG; r += kEpiThreads) {
+        const int k = r / N, h = r % N;
+        w_s[r] = (k < nm && h < a.H) ? (int32_t)__ldg(a.w + (int64_t)(q0 + k) * a.H + h) : 0;
+      }
+      if (et < QG) mpos[et] = et < nm ? __ldg(a.query_pos + q0 + et) : -1;
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bready);
       named_sync_epi();
-      if (et < a.H) {
+      for (int r = et; r < nm * a.H; r += kEpiThreads) {
+        const int k = r / a.H, h = r % a.H;
         int32_t sq = 0;
-        const int4* src = reinterpret_cast<const int4*>(qsrc + et * D);
+        const int4* src = reinterpret_cast<const int4*>(a.q + ((int64_t)(q0 + k) * a.H + h) * D);
         for (int c = 0; c < D / 16; ++c) {
           const int4 v = __ldg(src + c);
           const int32_t wv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
           for (int j = 0; j < 4; ++j)
 #pragma unroll
-            for (int b = 0; b < 4; ++b) sq += abs((int32_t)(int8_t)(wv[j] >> (8 * b)));
+            for (int b2 = 0; b2 < 4; ++b2) sq += abs((int32_t)(int8_t)(wv[j] >> (8 * b2)));
         }
-        const unsigned long long t = (unsigned long long)sq * (unsigned long long)abs(w_s[et]);
-        if (t) atomicAdd(bound_acc, t);
+        const unsigned long long t = (unsigned long long)sq * (unsigned long long)abs(w_s[k * N + h]);
+        if (t) atomicAdd(&bound_acc[k], t);
       }
     }
 
@@ -214,12 +273,12 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       if (lane == 0) {
         prefetch_tensormap(&kmap);
         const uint64_t pol = l2_policy_evict_first();
-        const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q) : q;
+        const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q0) : q0;
         int i = 0;
         for (; i < n_it; ++i) {
-          const int64_t g = git + i;
-          const int st = (int)(g % NST);
-          const uint32_t ph = (uint32_t)((g / NST) & 1);
+          const int64_t gi = git + i;
+          const int st = (int)(gi % NST);
+          const uint32_t ph = (uint32_t)((gi / NST) & 1);
           if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) break;
           const int32_t tile = tile0 + i;
           int64_t r[2];
@@ -228,7 +287,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           for (int j = 0; j < 2; ++j) {
             const int32_t p0 = tile * 128 + 64 * j;
             r[j] = -1;
-            if (p0 <= pos_q) {
+            if (p0 <= pos_hi) {
               r[j] = map_row(a.rows, seq, p0);
               if (r[j] < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
               else bytes += 64 * D;
@@ -250,23 +309,23 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
       if (lane == 0) {
-        constexpr uint32_t idesc = idesc_i8(128, N);
+        constexpr uint32_t idesc = idesc_i8(128, NG);
         const uint32_t b_addr = smem_u32(bmat);
         const bool bok = mbar_wait(bready, (uint32_t)(seg_count & 1), abort_flag);
         tc_fence_after();
         for (int i = 0; i < n_it && bok; ++i) {
-          const int64_t g = git + i;
-          const int st = (int)(g % NST);
-          const uint32_t ph = (uint32_t)((g / NST) & 1);
-          const int buf = (int)(g % NBUF);
-          const uint32_t tph = (uint32_t)((g / NBUF) & 1);
+          const int64_t gi = git + i;
+          const int st = (int)(gi % NST);
+          const uint32_t ph = (uint32_t)((gi / NST) & 1);
+          const int buf = (int)(gi % NBUF);
+          const uint32_t tph = (uint32_t)((gi / NBUF) & 1);
           if (!mbar_wait(&full[st], ph, abort_flag)) break;
           if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + st * TILE);
 #pragma unroll
           for (int k = 0; k < D / 32; ++k)
-            mma_i8(tmem_base + buf * N, smem_desc_kmajor(a_addr + 32 * k, D),
+            mma_i8(tmem_base + buf * NG, smem_desc_kmajor(a_addr + 32 * k, D),
                    smem_desc_kmajor(b_addr + 32 * k, D), idesc, k > 0 ? 1u : 0u);
           mma_commit(&empty[st]);
           mma_commit(&tfull[buf]);
@@ -276,58 +335,116 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       // ---------------------------------------------------------- epilogue
       // Two groups of four warps (one warp per TMEM lane quarter each) take
       // alternate tiles, so the groups never wait for each other within a
-      // segment.  A thread owns one key row: it loads the row's N head dots,
-      // frees the TMEM buffer, applies ReLU and the head weights (kept in
-      // registers) in independent partial sums, stores the score and adds
-      // its bucket to the shared histogram.  Every epilogue thread walks the
-      // same tiles and reaches the same barriers even after a timeout (it
-      // then skips the TMEM reads and the stores).
+      // segment.  A thread owns one key row: for each query of the segment's
+      // group it loads the row's N head dots, applies ReLU and the head
+      // weights in independent partial sums and stores the score (and, with
+      // one query per group, adds its bucket to the shared histogram); then
+      // it frees the TMEM buffer.  Every epilogue thread walks the same tiles
+      // and reaches the same barriers even after a timeout (it then skips the
+      // TMEM reads and the stores).
       if (seg_count == 0) pdl_wait();   // scores and histogram: after the grid before (it zeroes them)
-      constexpr bool kRegW = N <= 64;
+      constexpr bool kRegW = QG == 1 && N <= 64;
       int32_t wreg[kRegW ? N : 1];
       if constexpr (kRegW) {
 #pragma unroll
         for (int h = 0; h < N; ++h) wreg[h] = w_s[h];
       }
       for (int i = group; i < n_it; i += 2) {
-        const int64_t g = git + i;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[g % NBUF], (uint32_t)((g / NBUF) & 1), abort_flag));
-        uint32_t r[N];
-        if (ok) {
-          tc_fence_after();
-          const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((g % NBUF) * N);
-          if constexpr (N == 16) {
-            tmem_ld16(taddr, r);
-          } else {
+        const int64_t gi = git + i;
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[gi % NBUF], (uint32_t)((gi / NBUF) & 1), abort_flag));
+        const int32_t pos = (tile0 + i) * 128 + row;
+        if (ok) tc_fence_after();
+        const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)((gi % NBUF) * NG);
+        if constexpr (QG == 1) {
+          uint32_t r[N];
+          if (ok) {
+            if constexpr (N == 16) {
+              tmem_ld16(tbase, r);
+            } else {
 #pragma unroll
-            for (int c = 0; c < N / 32; ++c)
-              tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+              for (int c = 0; c < N / 32; ++c)
+                tmem_ld32(tbase + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * c]));
+            }
+            tmem_wait_ld();
           }
-          tmem_wait_ld();
+          tc_fence_before();   // the buffer has been read: free it for the MMA
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
+          if (ok) {
+            int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent chains, no long serial sum
+#pragma unroll
+            for (int h = 0; h < N; ++h) part[h & 7] += (kRegW ? wreg[h] : w_s[h]) * max((int32_t)r[h], 0);
+            const int32_t sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+            if (pos <= mpos[0]) {
+              a.scores[(int64_t)q0 * a.ld + pos] = sc;
+              atomicAdd(&hist_s[score_bucket(sc)], 1u);
+            }
+          }
+        } else {
+          // The group's N-column blocks (query k, head chunk c) are read 32 (or
+          // N) columns at a time, each load issued before the arithmetic of the
+          // block before it, so the TMEM latency overlaps the sums.
+          constexpr int CH = N < 32 ? N : 32;        // columns per block
+          constexpr int NCH = N / CH;                // blocks per query
+          const int nblk = nm * NCH;
+          uint32_t rb[2][CH];
+          auto ld_blk = [&](int bi, uint32_t (&dst)[CH]) {
+            const uint32_t ta = tbase + (uint32_t)((bi / NCH) * N + (bi % NCH) * CH);
+            if constexpr (CH == 16) tmem_ld16(ta, dst);
+            else tmem_ld32(ta, dst);
+          };
+          if (ok) {
+            ld_blk(0, rb[0]);
+            tmem_wait_ld();
+          }
+          int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+#pragma unroll 1
+          for (int bi = 0; bi < nblk; bi += 2) {
+#pragma unroll
+            for (int hb = 0; hb < 2; ++hb) {   // block bi + hb sits in rb[hb]
+              const int cur = bi + hb;
+              if (cur < nblk) {
+                if (ok && cur + 1 < nblk) ld_blk(cur + 1, rb[hb ^ 1]);
+                if (cur + 1 == nblk) {   // the buffer's last block is in registers: free it
+                  tc_fence_before();
+                  __syncwarp();
+                  if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
+                }
+                const int k = cur / NCH, c0 = (cur % NCH) * CH;
+                int4 wv[CH / 4];
+#pragma unroll
+                for (int u = 0; u < CH / 4; ++u) wv[u] = reinterpret_cast<const int4*>(w_s + k * N + c0)[u];
+                const int32_t* wp = reinterpret_cast<const int32_t*>(wv);
+#pragma unroll
+                for (int h = 0; h < CH; ++h) part[h & 7] += wp[h] * max((int32_t)rb[hb][h], 0);
+                if (c0 + CH == N) {   // query k is complete
+                  const int32_t sc =
+                      ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+#pragma unroll
+                  for (int z = 0; z < 8; ++z) part[z] = 0;
+                  if (ok && pos <= mpos[k]) a.scores[(int64_t)(q0 + k) * a.ld + pos] = sc;
+                }
+                if (ok && cur + 1 < nblk) tmem_wait_ld();
+              }
+            }
+          }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&tempty[g % NBUF]);
-        if (ok) {
-          int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};   // independent chains, no long serial sum
-#pragma unroll
-          for (int h = 0; h < N; ++h) part[h & 7] += (kRegW ? wreg[h] : w_s[h]) * max((int32_t)r[h], 0);
-          const int32_t sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-          const int32_t pos = (tile0 + i) * 128 + row;
-          if (pos <= pos_q) {
-            a.scores[(int64_t)q * a.ld + pos] = sc;
-            atomicAdd(&hist_s[score_bucket(sc)], 1u);
-          }
+        if (nm == 0) {   // no query (cannot happen for a segment with tiles): still free the buffer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
         }
       }
       // this query's histogram goes to global memory
       named_sync_epi();
-      if (a.hist) {
-        for (int b = et; b < kBuckets; b += kEpiThreads) {
-          const uint32_t v = hist_s[b];
-          if (v) {
-            atomicAdd(a.hist + (int64_t)q * kBuckets + b, v);
-            hist_s[b] = 0;
+      if constexpr (QG == 1) {
+        if (a.hist) {
+          for (int b2 = et; b2 < kBuckets; b2 += kEpiThreads) {
+            const uint32_t v = hist_s[b2];
+            if (v) {
+              atomicAdd(a.hist + (int64_t)q0 * kBuckets + b2, v);
+              hist_s[b2] = 0;
+            }
           }
         }
       }
@@ -336,8 +453,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     __syncthreads();   // the segment is done everywhere: B and the histogram may be reused
     tc_fence_after();
     if (tid == 64) {
-      if ((*bound_acc) * 128ull >= (1ull << 31)) record_error(a.status, CSA2_ERR_SCORE_RANGE);
-      *bound_acc = 0ull;
+      for (int k = 0; k < nm; ++k) {
+        if (bound_acc[k] * 128ull >= (1ull << 31)) record_error(a.status, CSA2_ERR_SCORE_RANGE);
+        bound_acc[k] = 0ull;
+      }
     }
     __syncthreads();
     git += n_it;
@@ -367,20 +486,22 @@ EncodeTiledFn encode_fn() {
 }
 
 template <int D>
-size_t index_smem_bytes(int N, int nq) {
+size_t index_smem_bytes(int N, int QG, int nq) {
   using Cfg = IndexCfg<D>;
-  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)N * D + kBuckets * 4 + 128 * 4 +
-         (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 + 32;
+  const int NG = N * QG;
+  return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)NG * D + (QG == 1 ? kBuckets * 4 : 0) +
+         (size_t)(NG > 128 ? NG : 128) * 4 + 2 * (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 +
+         32 + 8 * (size_t)QG + 4 * (size_t)QG + 16;
 }
 
-template <int D, int N>
+template <int D, int N, int QG>
 cudaError_t launch_one(const CUtensorMap& map, const IndexArgs& a, int grid, cudaStream_t st) {
-  const size_t smem = index_smem_bytes<D>(N, a.nq);
+  const size_t smem = index_smem_bytes<D>(N, QG, a.nq);
   static unsigned long long done = 0;
-  cudaError_t e = ensure_smem(index_score_kernel<D, N>, (int)index_smem_bytes<D>(N, kMaxQueries), done);
+  cudaError_t e = ensure_smem(index_score_kernel<D, N, QG>, (int)index_smem_bytes<D>(N, QG, kMaxQueries), done);
   if (e != cudaSuccess) return e;
-  return launch_k(index_score_kernel<D, N>, dim3(grid), dim3(64 + kEpiThreads), smem, st, false, launch_opts().pdl,
-                  map, a);
+  return launch_k(index_score_kernel<D, N, QG>, dim3(grid), dim3(64 + kEpiThreads), smem, st, false,
+                  launch_opts().pdl, map, a);
 }
 
 }  // namespace
@@ -395,7 +516,7 @@ cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st) {
+                               cudaStream_t st, bool* hist_built) {
   if (nq > kMaxQueries) return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -410,23 +531,28 @@ cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
 
-  IndexArgs a{q, w, seq_of_query, query_pos, to_rowmap(keys), nq, H, max_ctx, scores, ld, hist, status};
+  const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
+  // Many queries (a prefill chunk) share key tiles in groups of four, with the
+  // histogram left to the top-k; decode keeps one query per segment.
+  const bool grouped = nq >= kGroupMinQueries && N <= 64;
+  if (hist_built) *hist_built = !grouped && hist;
+  IndexArgs a{q, w, seq_of_query, query_pos, to_rowmap(keys), nq, H, max_ctx, scores, ld,
+              grouped ? nullptr : hist, status};
   const int64_t upper = (int64_t)nq * ((max_ctx + 127) / 128);
   const int grid = (int)(upper < sm_count() ? (upper > 0 ? upper : 1) : sm_count());
-  const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
   if (D == 128) {
     switch (N) {
-      case 16: return launch_one<128, 16>(map, a, grid, st);
-      case 32: return launch_one<128, 32>(map, a, grid, st);
-      case 64: return launch_one<128, 64>(map, a, grid, st);
-      default: return launch_one<128, 128>(map, a, grid, st);
+      case 16: return grouped ? launch_one<128, 16, 4>(map, a, grid, st) : launch_one<128, 16, 1>(map, a, grid, st);
+      case 32: return grouped ? launch_one<128, 32, 4>(map, a, grid, st) : launch_one<128, 32, 1>(map, a, grid, st);
+      case 64: return grouped ? launch_one<128, 64, 4>(map, a, grid, st) : launch_one<128, 64, 1>(map, a, grid, st);
+      default: return launch_one<128, 128, 1>(map, a, grid, st);
     }
   }
   switch (N) {
-    case 16: return launch_one<64, 16>(map, a, grid, st);
-    case 32: return launch_one<64, 32>(map, a, grid, st);
-    case 64: return launch_one<64, 64>(map, a, grid, st);
-    default: return launch_one<64, 128>(map, a, grid, st);
+    case 16: return grouped ? launch_one<64, 16, 4>(map, a, grid, st) : launch_one<64, 16, 1>(map, a, grid, st);
+    case 32: return grouped ? launch_one<64, 32, 4>(map, a, grid, st) : launch_one<64, 32, 1>(map, a, grid, st);
+    case 64: return grouped ? launch_one<64, 64, 4>(map, a, grid, st) : launch_one<64, 64, 1>(map, a, grid, st);
+    default: return launch_one<64, 128, 1>(map, a, grid, st);
   }
 }
 

@@ -87,12 +87,13 @@ size_t topk_scratch_bytes(int32_t nq, int32_t n_max);
 TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);
 
 // K1: scores of every visible position for every query (tcgen05 int8), plus
-// the bucket histogram.  hist may be NULL.
+// the bucket histogram.  hist may be NULL.  *hist_built (if given) says
+// whether the histogram was built: launches of many queries leave it out.
 cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st);
+                               cudaStream_t st, bool* hist_built = nullptr);
 
 // Radix top-k over score rows.  ks[0..n_k) are the wanted counts (n_k <= 2,
 // ks[0] >= ks[1]); outputs go to out_idx[t]/out_cnt[t].  If hist_ready, the
@@ -115,6 +116,16 @@ cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* 
                               const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                               int32_t* out_idx, int32_t* out_cnt, int32_t* status,
                               cudaStream_t st);
+
+// Exact top-k of many long rows (up to kRowSelMax candidates), one CTA per
+// row that builds its own histogram (topk_rows.cu).
+constexpr int kRowPer = 256;                  // candidates per thread
+constexpr int kRowSelMax = 1024 * kRowPer;    // per row
+cudaError_t launch_row_select(const int32_t* scores, int64_t ld, const int32_t* n_valid,
+                              const int32_t* query_pos, const int32_t* cand_pos, int32_t nq, int32_t n_max,
+                              const TopkOut* outs, int32_t n_k, int32_t* status, cudaStream_t st);
+// Whether launch_select can take these rows in one pass of co-resident CTAs.
+bool select_fits(int32_t nq, int32_t n_max);
 
 // Exact top-k of nq score rows in position order, for one or two k.  hist,
 // when given, is the complete bucket histogram of each row and s the scratch

@@ -21,6 +21,8 @@
 //   select  (topk_select.cu) when the rows fit on the device at once: the
 //           whole selection in one launch of co-resident CTAs; it is also the
 //           small-n path (n <= kSmallMax, one CTA per query)
+//   rows    (topk_rows.cu) many rows of up to kRowSelMax candidates: one CTA
+//           per row, with its own histogram
 // Otherwise, the multi-pass path:
 //   thresh  one CTA per query finds b* from the histogram
 //   gather  one CTA per 4096-candidate chunk counts the chunk's candidates
@@ -569,6 +571,10 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
   CandView v{scores, ld, n_valid, query_pos, cand_pos, n_max};
   const dim3 grid(s.n_chunks, nq);
   cudaError_t e;
+  // Many rows that do not fit on the device at once: one CTA per row, which
+  // builds its own histogram.
+  if (!select_fits(nq, n_max) && n_max <= kRowSelMax)
+    return launch_row_select(scores, ld, n_valid, query_pos, cand_pos, nq, n_max, outs, n_k, status, st);
   if (!hist_ready) {
     e = cudaMemsetAsync(s.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return e;

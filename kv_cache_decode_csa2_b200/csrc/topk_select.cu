@@ -337,6 +337,24 @@ SelDev g_sel_dev[64];
 
 }  // namespace
 
+bool select_fits(int32_t nq, int32_t n_max) {
+  if (n_max <= kSelSpan) return true;
+  const int64_t G = ((int64_t)n_max + kSelNT * 8 - 1) / (kSelNT * 8);
+  if (G > kSelMaxG) return false;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+  SelDev& d = g_sel_dev[dev];
+  if (!d.max_ctas) {
+    static unsigned long long done = 0;
+    int per_sm = 0;
+    if (ensure_smem(select_kernel<8>, kSelSmem, done) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<8>, kSelNT, kSelSmem) != cudaSuccess)
+      return false;
+    d.max_ctas = per_sm * sm_count();
+  }
+  return G * nq <= d.max_ctas;
+}
+
 cudaError_t launch_select(const int32_t* scores, int64_t ld, const int32_t* n_valid,
                           const int32_t* query_pos, const int32_t* cand_pos, int32_t nq, int32_t n_max,
                           const TopkOut* outs, int32_t n_k, const uint32_t* hist, const TopkScratch* s,

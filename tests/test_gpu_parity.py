@@ -157,6 +157,41 @@ def test_topk_pool_matches_oracle(n, k, spread):
         assert (o[i, c[i]:] == -1).all()
 
 
+@pytest.mark.parametrize("spread,k", [(10 ** 6, 700), (1000, 512), (2, 600), (0, 512)])
+def test_topk_many_long_rows(spread, k):
+    """40 rows of up to 50,000 candidates: more rows than fit on the device at
+    once, so every row gets one CTA.  Spread 2 and 0 make the tie list too
+    long to rank (radix path); ragged valid counts include one below k."""
+    rng = np.random.default_rng(spread + k)
+    nq, n = 40, 50000
+    s = rng.integers(-spread, spread + 1, size=(nq, n)).astype(np.int32)
+    nv = rng.integers(n // 2, n + 1, size=nq).astype(np.int32)
+    nv[3] = k // 2
+    out = torch.empty((nq, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((nq,), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_topk_pool(torch.from_numpy(s).to(DEV), k, out, out_cnt=cnt,
+                                    n_valid=torch.from_numpy(nv).to(DEV)))
+    o, c = _np(out), _np(cnt)
+    for i in range(nq):
+        ref = O.top_k_positions(s[i, :nv[i]], np.arange(nv[i]), k)
+        assert c[i] == len(ref) and np.array_equal(o[i, :c[i]], ref), f"row {i}"
+        assert (o[i, c[i]:] == -1).all()
+
+
+def test_topk_many_long_rows_with_positions():
+    rng = np.random.default_rng(9)
+    nq, n = 24, 70000
+    s = rng.integers(0, 50, size=(nq, n)).astype(np.int32)
+    pos = np.sort(rng.choice(10 ** 7, size=(nq, n), replace=True), axis=1).astype(np.int32)
+    pos += np.arange(n, dtype=np.int32)[None]          # strictly ascending per row
+    out = torch.empty((nq, 512), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_topk_pool(torch.from_numpy(s).to(DEV), 512, out,
+                                    cand_pos=torch.from_numpy(pos).to(DEV)))
+    o = _np(out)
+    for i in range(nq):
+        assert np.array_equal(o[i], O.top_k_positions(s[i], pos[i], 512)), f"row {i}"
+
+
 @pytest.mark.parametrize("n", [1000, 16000, 40000])
 def test_topk_all_equal_and_two_valued(n):
     for s in (np.zeros((1, n), np.int32), np.where(np.arange(n) % 3 == 0, 7, -7).astype(np.int32)[None]):

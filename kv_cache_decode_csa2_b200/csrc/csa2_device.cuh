@@ -246,6 +246,21 @@ __host__ __device__ __forceinline__ uint32_t score_bucket(int32_t s) {
   return s >= 0 ? 4096u + score_f((uint32_t)s) : 4095u - score_f((uint32_t)(-(s + 1)));
 }
 constexpr int kBuckets = 8192;
+// The smallest score whose bucket is >= b (the bucket is monotone in the
+// score), by binary search; INT32_MAX if no score reaches bucket b, and
+// INT32_MIN for b <= 0.
+__host__ __device__ __forceinline__ int32_t bucket_min_score(int32_t b) {
+  if (b <= 0) return INT32_MIN;
+  if (b >= kBuckets) return INT32_MAX;
+  int64_t lo = INT32_MIN, hi = INT32_MAX;   // invariant: bucket(hi) >= b
+  if ((int32_t)score_bucket(INT32_MAX) < b) return INT32_MAX;
+  while (lo + 1 < hi) {
+    const int64_t mid = lo + (hi - lo) / 2;
+    if ((int32_t)score_bucket((int32_t)mid) >= b) hi = mid;
+    else lo = mid;
+  }
+  return (int32_t)hi;
+}
 
 // Ordering key of a candidate: larger key = better (higher score, then lower
 // position).  All keys of distinct positions differ.

@@ -5,8 +5,10 @@
 // context has 2048 rows of up to 262,144 candidates: far more rows than the
 // select kernel can hold co-resident.  Here one CTA of kRowNT threads takes a
 // row, and thread t owns the candidates [t R, t R + R), R <= kRowPer:
-//   pass 1  bucket histogram of the row in shared memory; one block scan
-//           finds the threshold bucket b* of each target;
+//   pass 1  bucket histogram of the row in shared memory, counting only
+//           candidates at or above a cut that a small sample of the row
+//           picks (with a full-histogram redo should too few clear it); one
+//           block scan finds the threshold bucket b* of each target;
 //   pass 2  per-thread bitmasks of the members above b* and of the ties at
 //           b*; the ties go to a shared list, each warp ranks some of them
 //           against it, and this gives the smallest member tie key;
@@ -98,42 +100,21 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     for (; j < j1; ++j) f(j, __ldcg(row + j));
   };
 
-  // ---- pass 1: histogram, threshold buckets
-  {
+  // ---- pass 1: histogram, threshold buckets.  A sample (each thread's first
+  // 8 candidates) picks a lower cut that about four times the wanted count
+  // clears; the exact histogram then counts only candidates at or above it,
+  // which spares most shared-memory atomics.  Should fewer than k candidates
+  // clear the cut, the full histogram is built instead.
+  __shared__ int32_t cut_s;
+  const int32_t kmax = n_k > 1 && a.k[1] > a.k[0] ? a.k[1] : a.k[0];
+  auto zero_hist = [&]() {
     uint4* h4 = reinterpret_cast<uint4*>(hist + tid * 8);
     h4[0] = make_uint4(0, 0, 0, 0);
     h4[1] = make_uint4(0, 0, 0, 0);
-  }
-  __syncthreads();
-  // pass 1 over words of 32 candidates; a word's eight loads are all issued
-  // before any is used, so the memory latency is paid once per word
-#pragma unroll 1
-  for (int x = 0; x < kRowWords; ++x) {
-    const int32_t base = j0 + 32 * x;
-    if (base >= j1) break;
-    if (vec && base + 32 <= j1) {
-      int4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const int4*>(row + base) + u);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        atomicAdd(&hist[score_bucket(v[u].x)], 1u);
-        atomicAdd(&hist[score_bucket(v[u].y)], 1u);
-        atomicAdd(&hist[score_bucket(v[u].z)], 1u);
-        atomicAdd(&hist[score_bucket(v[u].w)], 1u);
-      }
-    } else {
-      for (int e = 0; e < 32 && base + e < j1; ++e) atomicAdd(&hist[score_bucket(__ldcg(row + base + e))], 1u);
-    }
-  }
-  if (a.cand_pos) {   // candidate positions must ascend
-    const int32_t* cp = a.cand_pos + (int64_t)q * a.ld;
-    bool bad = false;
-    for (int32_t j = j0 > 0 ? j0 : 1; j < j1; ++j) bad |= __ldg(cp + j) <= __ldg(cp + j - 1);
-    if (bad) record_error(a.status, CSA2_ERR_ORDER);
-  }
-  __syncthreads();
-  {
+  };
+  // walks this thread's 8 bins for the bucket where the count above crosses
+  // `want`; returns the block total
+  auto scan_bins = [&](auto&& on_cross) -> int64_t {
     const uint4* h4 = reinterpret_cast<const uint4*>(hist + tid * 8);
     const uint4 h0 = h4[0], h1 = h4[1];
     const uint32_t hb[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
@@ -142,28 +123,124 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     for (int b = 0; b < 8; ++b) hsum += hb[b];
     uint64_t total64;
     const uint64_t excl = sel_scan<kRowNT>(hsum, wtmp, &total64);
-    const int64_t total = (int64_t)total64, above_me = total - (int64_t)excl - hsum;
+    const int64_t above_me = (int64_t)total64 - (int64_t)excl - hsum;
+    on_cross(hb, above_me, hsum, (int64_t)total64);
+    return (int64_t)total64;
+  };
+  zero_hist();
+  if (tid == 0) cut_s = -1;
+  __syncthreads();
+  if (n > kmax) {   // the sample
+    const int32_t m = j1 - j0 < 8 ? j1 - j0 : 8;
+    int32_t v[8];
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int32_t k = a.k[t];
-      if (t < n_k && total > k && above_me < k && above_me + hsum >= k) {
+    for (int e = 0; e < 8; ++e) v[e] = e < m ? __ldcg(row + j0 + e) : 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (e < m) atomicAdd(&hist[score_bucket(v[e])], 1u);
+  }
+  __syncthreads();
+  if (n > kmax) {
+    scan_bins([&](const uint32_t (&hb)[8], int64_t above_me, uint32_t hsum, int64_t S) {
+      const int64_t want = 4 * (int64_t)kmax * S / n + 16;   // S samples of n candidates
+      if (above_me < want && above_me + hsum >= want) {
         int64_t acc = above_me;
 #pragma unroll
         for (int b = 7; b >= 0; --b) {
-          if (acc + hb[b] >= k) {
-            bstar_s[t] = tid * 8 + b;
-            above_s[t] = (int32_t)acc;
+          if (acc + hb[b] >= want) {
+            cut_s = tid * 8 + b;
             break;
           }
           acc += hb[b];
         }
       }
+    });
+  }
+  zero_hist();
+  __shared__ int32_t cut_score_s;
+  if (tid == 0) cut_score_s = bucket_min_score(cut_s);
+  __syncthreads();
+  const int32_t cut_score = cut_score_s;
+#pragma unroll 1
+  for (int attempt = 0; attempt < 2; ++attempt) {
+    const int32_t lo_s = attempt == 0 ? cut_score : INT32_MIN;   // count scores >= lo_s
+    // words of 32 candidates; a word's eight loads are all issued before any is used
+#pragma unroll 1
+    for (int x = 0; x < kRowWords; ++x) {
+      const int32_t base = j0 + 32 * x;
+      if (base >= j1) break;
+      if (vec && base + 32 <= j1) {
+        int4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const int4*>(row + base) + u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int32_t sv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (sv[e] >= lo_s) atomicAdd(&hist[score_bucket(sv[e])], 1u);
+        }
+      } else {
+        for (int e = 0; e < 32 && base + e < j1; ++e) {
+          const int32_t sv = __ldcg(row + base + e);
+          if (sv >= lo_s) atomicAdd(&hist[score_bucket(sv)], 1u);
+        }
+      }
     }
+    if (attempt == 0 && a.cand_pos) {   // candidate positions must ascend
+      const int32_t* cp = a.cand_pos + (int64_t)q * a.ld;
+      bool bad = false;
+      for (int32_t j = j0 > 0 ? j0 : 1; j < j1; ++j) bad |= __ldg(cp + j) <= __ldg(cp + j - 1);
+      if (bad) record_error(a.status, CSA2_ERR_ORDER);
+    }
+    __syncthreads();
+    const int64_t total = scan_bins([&](const uint32_t (&hb)[8], int64_t above_me, uint32_t hsum, int64_t) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int32_t k = a.k[t];
+        if (t < n_k && n > k && above_me < k && above_me + hsum >= k) {
+          int64_t acc = above_me;
+#pragma unroll
+          for (int b = 7; b >= 0; --b) {
+            if (acc + hb[b] >= k) {
+              bstar_s[t] = tid * 8 + b;
+              above_s[t] = (int32_t)acc;
+              break;
+            }
+            acc += hb[b];
+          }
+        }
+      }
+    });
+    // the counted candidates must cover every target that is not "take all"
+    bool short_of = false;
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+      if (t < n_k && n > a.k[t] && total < a.k[t]) short_of = true;
+    if (!short_of) break;
+    zero_hist();
+    if (tid < 2) {
+      bstar_s[tid] = -1;
+      above_s[tid] = 0;
+    }
+    __syncthreads();
   }
   __syncthreads();
 
   // ---- pass 2: members above b* and ties at b*, as bitmasks
   const int32_t b0 = bstar_s[0], b1 = n_k > 1 ? bstar_s[1] : INT32_MIN;
+  // score ranges: above b* means s >= hi_t, at b* means lo_t <= s < hi_t
+  // (64-bit: the bucket above the top one starts past every int32 score)
+  __shared__ long long bound_s[4];
+  if (tid < 4) {
+    const int t = tid >> 1;
+    const int32_t bs = bstar_s[t];
+    const int32_t b = (tid & 1) ? bs + 1 : bs;
+    bound_s[tid] = (t >= n_k || bs < 0) ? 0ll : b >= kBuckets ? (long long)INT32_MAX + 1 : bucket_min_score(b);
+  }
+  __syncthreads();
+  const long long lo0 = bound_s[0], hi0 = bound_s[1], lo1 = bound_s[2], hi1 = bound_s[3];
+  const bool all0 = b0 < 0, all1 = n_k > 1 && b1 < 0;
   uint32_t above_m[NK][kRowWords], tie_m[NK][kRowWords];
 #pragma unroll
   for (int t = 0; t < NK; ++t)
@@ -176,14 +253,15 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     if (base < j1) {
       auto take = [&](int e, int32_t s) {
         const uint32_t bit = 1u << e;
-        const int32_t bk = (int32_t)score_bucket(s);
-        if (bk > b0) above_m[0][x] |= bit;   // b* = -1 takes every candidate
-        if (NK > 1 && bk > b1) above_m[NK - 1][x] |= bit;
-        if (bk == b0 || bk == b1) {
+        if (all0 || s >= hi0) above_m[0][x] |= bit;   // b* = -1 takes every candidate
+        if (NK > 1 && (all1 || s >= hi1)) above_m[NK - 1][x] |= bit;
+        const bool t0 = !all0 && s >= lo0 && s < hi0;
+        const bool t1 = NK > 1 && !all1 && s >= lo1 && s < hi1;
+        if (t0 || t1) {
           const uint64_t key = cand_key(s, base + e);
 #pragma unroll
           for (int t = 0; t < NK; ++t) {
-            if (bk == (t ? b1 : b0)) {
+            if (t ? t1 : t0) {
               tie_m[t][x] |= bit;
               const uint32_t slot = atomicAdd(&nt_s[t], 1u);
               if (slot < (uint32_t)kRowTieCap) ties[t * kRowTieCap + slot] = key;

@@ -17,6 +17,15 @@ prints one JSON line.
 
 --impl reference times the CPU oracle (oracle/) on the same workload, on this
 host's cores; there is no other reference implementation of this path.
+
+    python bench.py --workload prefill [--steps K] [--warmup W]
+
+times the prefill-chunk configuration instead: 2048 causal queries at
+positions 260096-262143 of a 262,144-row context, each scoring its whole
+prefix with the int8 indexer, keeping its top-512 and attending to them plus
+the 128-row window (one csa2_index_full and one csa2_sparse_attn_fp4 call,
+captured in a CUDA graph per replica).  It prints queries/s and the int8
+TOP/s of the index stage.
 """
 from __future__ import annotations
 
@@ -40,6 +49,12 @@ import synth  # noqa: E402
 
 METRIC = "decode steps/s and HBM GB/s (% of B200 roofline) at 1M-token context"
 WL = synth.C2_1M_PLAN
+METRIC_PREFILL = "prefill-chunk queries/s and index int8 TOP/s (2048 causal queries, 262144 context)"
+WL_PREFILL = synth.C4_PREFILL
+# DRAM bytes (read + write) of one index-score launch on the decode workload,
+# from one ncu capture of this kernel on it (its summary is kept with the
+# profiles); to be reset to None whenever that kernel changes.
+K1_TRAFFIC_BYTES = 134_273_792 + 4_593_664
 N_REPLICAS = 4
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 NOMINAL_HBM_GBS = 8000.0
@@ -487,7 +502,7 @@ def run_gpu(args, rank, world, local):
             "roofline": {"kernel": "index_score_kernel<128,64> (full-mode index scoring of 1M keys)",
                          "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"], "ms_per_launch": k_ms,
-                         "bytes_per_launch": key_bytes, "traffic": None},
+                         "bytes_per_launch": key_bytes, "traffic": K1_TRAFFIC_BYTES},
             "e2e": {"value": e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d_bytes,
                     "d2h_bytes_per_step": d2h_bytes, "path": "pinned H2D + csa2_layer_plan + D2H, no graph"},
             "gpu_launches": kernels_per_step(wl) * args.steps,
@@ -503,6 +518,213 @@ def run_gpu(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- prefill chunk
+def peak_int8_tops() -> dict:
+    """Dense int8 tensor peak: the measured bf16 GEMM rate times the nominal
+    int8/bf16 ratio (4.5 / 2.25 PFLOP/s); the fallback bf16 figure if the
+    measured file is absent."""
+    try:
+        with open(PEAKS_FILE) as f:
+            bf16 = float(json.load(f)["bf16_tflops"])
+        return {"tops": 2.0 * bf16, "src": "measured bf16 x 2 (nominal int8/bf16 ratio)"}
+    except Exception:
+        return {"tops": 2.0 * 1590.0, "src": "fallback bf16 x 2 (nominal int8/bf16 ratio)"}
+
+
+def prefill_replica(wl, host, dev, status):
+    """Device state of one prefill chunk: keys, FP4 cache, the queries."""
+    from kv_cache_decode_csa2_b200 import csa2 as B
+    n, q, w, qa = host
+    codes = torch.empty((n, wl.attn_dim // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, wl.attn_dim // 32), dtype=torch.uint8, device=dev)
+    step = 1 << 17
+    for a in range(0, n, step):                # FP4 cache written by the library's quantiser
+        b = min(n, a + step)
+        x = torch.from_numpy(synth.kv_values(wl, 0, 0, a, b)).to(dev)
+        B.csa2_fp4_quantize(x, codes[a:b], scales[a:b], status=status)
+    keys = torch.from_numpy(synth.index_keys(wl, 0, 0)).to(dev)
+    return {"keys": B.Rows(keys), "codes": B.Rows(codes), "scales": B.Rows(scales),
+            "q": torch.from_numpy(q).to(dev), "w": torch.from_numpy(w).to(dev),
+            "qa": torch.from_numpy(qa).to(dev).to(torch.bfloat16)}
+
+
+PREFILL_SAMPLE = "the chunk's last query (its whole 262,144-row prefix), through the oracle one query at a time"
+
+
+def prefill_host(wl):
+    n = int(wl.lengths()[0])
+    _, qp = wl.query_positions()
+    qs = [synth.index_query(wl, 0, i) for i in range(len(qp))]
+    return (n, np.stack([x[0] for x in qs]), np.stack([x[1] for x in qs]),
+            np.stack([synth.attn_query(wl, 0, i) for i in range(len(qp))]))
+
+
+def oracle_prefill_query_seconds(wl, host, qp) -> float:
+    """Seconds the oracle takes for one query of the chunk (the last, whose
+    prefix is the whole context): its scores, its top-k and its attention.
+    The FP4 rows of its attention set are stored, untimed, in between."""
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+    keys = synth.index_keys(wl, 0, 0)
+    i = len(qp) - 1
+    pos = int(qp[i])
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        s_ = O.index_scores(host[1][i], host[2][i], keys[:pos + 1])
+        sel_ = O.top_k_positions(s_, np.arange(pos + 1), wl.topk)
+        S = O.attention_set(sel_, pos, wl.window)
+        t1 = time.perf_counter()
+        x = np.concatenate([synth.kv_values(wl, 0, 0, int(r_), int(r_) + 1) for r_ in S])
+        c_, sc_ = O.fp4_quantize(x)
+        t2 = time.perf_counter()
+        O.sparse_attention(host[3][i], O.fp4_dequant(c_, sc_, wl.attn_dim))
+        t3 = time.perf_counter()
+    return (t1 - t0) + (t3 - t2)
+
+
+def run_reference_prefill(args, rank, world):
+    if rank != 0:
+        return
+    wl = WL_PREFILL
+    host = prefill_host(wl)
+    _, qp = wl.query_positions()
+    ts = [oracle_prefill_query_seconds(wl, host, qp) for _ in range(max(1, min(args.steps, 3)))]
+    v = 1.0 / (sum(ts) / len(ts))
+    line = {"impl": "reference", "metric": METRIC_PREFILL, "value": v, "unit": "queries/s", "n_gpus": args.gpus,
+            "steps": len(ts), "warmup": 0, "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64,f64", "data": "synthetic",
+            "config": {"workload": wl.name},
+            "cpu_baseline": {"value": v, "unit": "queries/s", "cores": cpu_cores_used(), "kind": "oracle",
+                             "sample": PREFILL_SAMPLE},
+            "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_prefill(args, rank, world, local):
+    from kv_cache_decode_csa2_b200 import csa2 as B
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    wl = WL_PREFILL
+    t_setup = time.time()
+    sq, qp = wl.query_positions()
+    nq = len(qp)
+    host = prefill_host(wl)
+    n = host[0]
+    status = B.new_status(dev)
+    n_rep = max(1, args.replicas)
+    reps = [prefill_replica(wl, host, dev, status) for _ in range(n_rep)]
+    pos_dev = torch.from_numpy(qp.astype(np.int32)).to(dev)
+    seq_dev = torch.from_numpy(sq.astype(np.int32)).to(dev)
+    sel = torch.empty((nq, wl.topk), dtype=torch.int32, device=dev)
+    cnt = torch.empty((nq,), dtype=torch.int32, device=dev)
+    out = torch.empty((nq, wl.attn_heads, wl.attn_dim), dtype=torch.bfloat16, device=dev)
+    L = B.lib()
+    ws_i = torch.empty(L.csa2_index_full_workspace(nq, n, 0, wl.topk), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(L.csa2_sparse_attn_workspace(nq, wl.attn_heads, wl.attn_dim, wl.topk, wl.window),
+                       dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def index(r):
+        B.csa2_index_full(r["q"], r["w"], r["keys"], pos_dev, n, seq_of_query=seq_dev, K=wl.topk, sel_idx=sel,
+                          sel_cnt=cnt, status=status, ws=ws_i, stream=stream)
+
+    def attend(r):
+        B.csa2_sparse_attn_fp4(r["qa"], r["codes"], r["scales"], pos_dev, sel, out, sel_cnt=cnt,
+                               seq_of_query=seq_dev, window=wl.window, status=status, ws=ws_a, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for r in reps:                         # ordinary calls first (one-time kernel set-up)
+            index(r)
+            attend(r)
+    torch.cuda.synchronize()
+    B.check_status(status)
+    graphs, igraphs = [], []
+    for r in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            index(r)
+            attend(r)
+        graphs.append(g)
+        gi = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gi, stream=stream):
+            index(r)
+        igraphs.append(gi)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t_setup
+
+    def timed(gs, steps):
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                gs[i % n_rep].replay()
+        torch.cuda.synchronize()
+        barrier(world)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for i in range(steps):
+                gs[i % n_rep].replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), world, dev) / steps
+
+    with ClockSampler(gpu_id(dev)) as clk:
+        time.sleep(0.3)
+        ms = timed(graphs, args.steps)
+    ms_index = timed(igraphs, max(3, args.steps))
+    B.check_status(status)
+    ops = sum((int(p) + 1) * wl.idx_heads * wl.idx_dim * 2 for p in qp)
+    tops = ops / (ms_index / 1e3) / 1e12
+    pk = peak_int8_tops()
+
+    # end to end: the chunk's queries in from pinned host memory, outputs back
+    r0 = reps[0]
+    h2d = [r0["q"], r0["w"], r0["qa"]]
+    h2d_host = [t.cpu().pin_memory() for t in h2d]
+    d2h = [out, sel]
+    d2h_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d2h]
+    e_steps = max(3, args.steps // 2)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e_steps):
+            for hsrc, ddst in zip(h2d_host, h2d):
+                ddst.copy_(hsrc, non_blocking=True)
+            index(r0)
+            attend(r0)
+            for dsrc, hdst in zip(d2h, d2h_host):
+                hdst.copy_(dsrc, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e_steps
+    B.check_status(status)
+
+    line = {"metric": METRIC_PREFILL, "value": world * nq / (ms / 1e3), "unit": "queries/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": {"workload": wl.name, "ctx": n, "queries": nq, "first_pos": int(qp[0]), "topk": wl.topk,
+                       "window": wl.window, "indexer": f"int8 {wl.idx_heads}x{wl.idx_dim}, w int8",
+                       "kv": f"FP4 E2M1 d{wl.attn_dim}, E4M3 per 32", "q_heads": wl.attn_heads,
+                       "l2": f"inputs rotate over {n_rep} device replicas (~180 MB each)",
+                       "parallelism": "one chunk per rank"},
+            "roofline": {"kernel": "index stage: index_score_kernel<128,64,4> + per-query top-512",
+                         "bound": "tensor", "achieved": tops, "peak": pk["tops"], "unit": "TOP/s (int8)",
+                         "frac": tops / pk["tops"], "peak_src": pk["src"], "ms_per_launch": ms_index,
+                         "ops_per_launch": ops, "traffic": None},
+            "e2e": {"value": world * nq / (e_ms / 1e3), "unit": "queries/s",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h2d_host),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in d2h_host),
+                    "path": "pinned H2D + csa2_index_full + csa2_sparse_attn_fp4 + D2H, no graph"},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
+    if rank == 0 and not args.no_cpu_baseline:
+        sec = oracle_prefill_query_seconds(wl, host, qp)
+        line["cpu_baseline"] = {"value": 1.0 / sec, "unit": "queries/s", "cores": cpu_cores_used(), "kind": "oracle",
+                                "sample": PREFILL_SAMPLE}
+    del graphs, igraphs
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -510,6 +732,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: the 1M-context 8-layer step (default); prefill: the 2048-query chunk")
     ap.add_argument("--replicas", type=int, default=N_REPLICAS,
                     help="device copies of the state rotated between steps (4 keep each step's reads out of L2)")
     args = ap.parse_args()
@@ -517,7 +741,10 @@ def main():
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_init(args.gpus)
     try:
-        if args.impl == "reference":
+        if args.workload == "prefill":
+            (run_reference_prefill if args.impl == "reference" else run_prefill)(args, rank, world, *(
+                () if args.impl == "reference" else (local,)))
+        elif args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_gpu(args, rank, world, local)

@@ -100,12 +100,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int warp = tid >> 5;
   const int lane = tid & 31;
 
-  // ---- groups: runs of consecutive queries of one sequence, cut every QG
-  for (int i = tid; i < a.nq; i += blockDim.x) {
-    const int32_t pos = __ldg(a.query_pos + i);
-    if (pos < 0 || pos >= a.max_ctx) record_error(a.status, CSA2_ERR_INDEX_RANGE);
-  }
-  for (int i = tid; i < kHist; i += blockDim.x) hist_s[i] = 0;
+  // ---- prologue: warp 0 builds the work list (groups of queries and the
+  // tiles before each group), warp 1 allocates TMEM, thread 0 sets up the
+  // barriers; one block barrier later the producer streams.  The epilogue
+  // warps zero their histogram behind a barrier of their own.
   if (tid == 0) {
     for (int i = 0; i < NST; ++i) {
       mbar_init(&full[i], 1);
@@ -125,11 +123,14 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     tmem_relinquish();
   }
   if (warp == 0) {
+    // groups: runs of consecutive queries of one sequence, cut every QG
+    int32_t n_groups = 0;
     if constexpr (QG == 1) {
       for (int i = lane; i <= a.nq; i += 32) gq[i] = i;
-      if (lane == 0) *ngroups_s = a.nq;
+      n_groups = a.nq;
+      __syncwarp();
     } else {
-      int32_t last_start = 0, n_groups = 0;
+      int32_t last_start = 0;
       for (int base = 0; base < a.nq; base += 32) {
         const int i = base + lane;
         const bool valid = i < a.nq;
@@ -152,36 +153,32 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
         n_groups += __popc(bal);
         last_start = __shfl_sync(0xffffffffu, v, 31);
       }
-      if (lane == 0) {
-        gq[n_groups] = a.nq;
-        *ngroups_s = n_groups;
-      }
+      if (lane == 0) gq[n_groups] = a.nq;
+      __syncwarp();
     }
-  }
-  __syncthreads();
-  const int ngroups = *ngroups_s;
-  // prefix[g+1] = tiles of group g: the longest causal prefix of its queries
-  for (int g = tid; g < ngroups; g += blockDim.x) {
-    int32_t t = 0;
-    for (int i = gq[g]; i < gq[g + 1]; ++i) {
-      const int32_t pos = __ldg(a.query_pos + i);
-      if (pos >= 0 && pos < a.max_ctx && (pos + 128) / 128 > t) t = (pos + 128) / 128;
-    }
-    prefix[g + 1] = t;
-  }
-  if (tid == 0) prefix[0] = 0;
-  __syncthreads();
-  if (warp == 0) {   // inclusive scan of tile counts, 32 at a time
+    // prefix[g+1] = tiles up to group g: a group's tiles cover the longest
+    // causal prefix of its queries
     int32_t carry = 0;
-    for (int base = 0; base < ngroups; base += 32) {
-      const int i = base + lane;
-      int32_t v = (i < ngroups) ? prefix[i + 1] : 0;
+    if (lane == 0) {
+      prefix[0] = 0;
+      *ngroups_s = n_groups;
+    }
+    for (int base = 0; base < n_groups; base += 32) {
+      const int g = base + lane;
+      int32_t v = 0;
+      if (g < n_groups) {
+        for (int i = gq[g]; i < gq[g + 1]; ++i) {
+          const int32_t pos = __ldg(a.query_pos + i);
+          if (pos < 0 || pos >= a.max_ctx) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+          else if ((pos + 128) / 128 > v) v = (pos + 128) / 128;
+        }
+      }
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += n;
       }
-      if (i < ngroups) prefix[i + 1] = v + carry;
+      if (g < n_groups) prefix[g + 1] = v + carry;
       carry += __shfl_sync(0xffffffffu, v, 31);
     }
   }
@@ -189,7 +186,12 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const int ngroups = *ngroups_s;
   pdl_trigger();   // the next grid may be launched (it waits for this one to finish)
+  if (warp >= 2) {   // the epilogue's histogram, zeroed before its first use
+    for (int i = tid - 64; i < kHist; i += kEpiThreads) hist_s[i] = 0;
+    named_sync_epi();
+  }
 
   const int64_t total = prefix[ngroups];
   const int64_t lo = total * blockIdx.x / gridDim.x;

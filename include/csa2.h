@@ -120,7 +120,13 @@ typedef struct csa2_rows {
  *   K, sel_idx, sel_cnt     K > 0: int32 [nq][K] the K best positions (the
  *                           top-K of the pool under the same scores, i.e. the
  *                           global top-K) and their count
- * Supported: D in {64, 128}; 1 <= H <= 128; nq >= 1; P, K in [0, 65536].
+ * Every query scores its own causal prefix 0..query_pos[i], so a prefill
+ * chunk (many queries of one sequence at consecutive positions) is one call;
+ * with P = 0 and K > 0 each query keeps its top-K of the whole prefix.  From
+ * 16 queries on, consecutive queries of one sequence share key tiles in
+ * groups of four.
+ * Supported: D in {64, 128}; 1 <= H <= 128; 1 <= nq <= 4096; P, K in
+ * [0, 65536].
  * Errors on the device: SCORE_RANGE, INDEX_RANGE.
  */
 int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,

@@ -118,6 +118,7 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
                         int32_t* status, void* stream) {
   if (!q || !w || !query_pos || !status || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
   if (nq < 1 || max_ctx < 1 || P < 0 || K < 0 || P > 65536 || K > 65536) return CSA2_ERR_INVALID_ARG;
+  if (nq > 4096) return CSA2_ERR_UNSUPPORTED;   // the index-score kernel's work list holds 4096 queries
   if (D != 64 && D != 128) return CSA2_ERR_UNSUPPORTED;
   if (H < 1 || H > 128 || nq > 4096) return CSA2_ERR_UNSUPPORTED;
   if (!rows_ok(keys, D, 16)) return CSA2_ERR_INVALID_ARG;

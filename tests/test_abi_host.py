@@ -80,6 +80,9 @@ def test_rejects_bad_arguments_before_any_launch():
     # workspace too small
     assert L.csa2_index_full(16, 16, ctypes.byref(keys), None, 16, 1, 64, 128, 10, None, 0, 0, None, None,
                              0, None, None, 256, 8, 16, None) == 3
+    # more queries than one launch's work list holds
+    assert L.csa2_index_full(16, 16, ctypes.byref(keys), None, 16, 4097, 64, 128, 10, None, 0, 0, None, None,
+                             0, None, None, 256, 1 << 20, 16, None) == 2
     # top-k: k out of range
     assert L.csa2_topk_pool(16, 10, None, None, 1, 10, 0, 16, None, None, 0, 16, None) == 1
     # reindex: K > P

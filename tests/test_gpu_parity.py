@@ -280,6 +280,37 @@ def test_reindex_batch_of_many_queries():
         assert np.array_equal(sels[i, :len(ref_sel)], ref_sel)
 
 
+def test_index_grouped_queries_of_several_sequences():
+    """20 queries over three sequences (runs of 7, 1 and 12 queries): from 16
+    queries on, consecutive queries of one sequence share key tiles in groups
+    of at most four, so this has partial and single-query groups.  Every
+    query's scores and its top-K of the whole prefix must equal the oracle's."""
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(9000, 5000, 12000), modes=(synth.FULL,))
+    lens = wl.lengths()
+    seq = np.array([0] * 7 + [1] + [2] * 12, dtype=np.int32)
+    pos = np.concatenate([np.arange(8990, 8997), [4999], np.arange(11900, 12000, 9)[:12]]).astype(np.int32)
+    keys_host = [synth.index_keys(wl, 0, s_) for s_ in range(len(lens))]
+    kt, srows = G._place(keys_host, lens, None, 64, wl.idx_dim, np.int8, DEV)
+    keys = B.Rows(kt, None, 64, srows)
+    qs = [synth.index_query(wl, 0, i) for i in range(len(pos))]
+    q = torch.from_numpy(np.stack([x[0] for x in qs])).to(DEV)
+    w = torch.from_numpy(np.stack([x[1] for x in qs])).to(DEV)
+    nq, K = len(pos), 300
+    max_ctx = int(lens.max())
+    scores = torch.full((nq, max_ctx), -7, dtype=torch.int32, device=DEV)
+    sel = torch.empty((nq, K), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((nq,), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_index_full(q, w, keys, torch.from_numpy(pos).to(DEV), max_ctx,
+                                     seq_of_query=torch.from_numpy(seq).to(DEV), scores=scores, K=K,
+                                     sel_idx=sel, sel_cnt=cnt))
+    sc, so, co = _np(scores), _np(sel), _np(cnt)
+    for i in range(nq):
+        ref = O.index_scores(qs[i][0], qs[i][1], keys_host[seq[i]][:pos[i] + 1])
+        assert np.array_equal(sc[i, :pos[i] + 1], ref), f"query {i} scores"
+        ref_sel = O.top_k_positions(ref, np.arange(pos[i] + 1), K)
+        assert co[i] == len(ref_sel) and np.array_equal(so[i, :co[i]], ref_sel), f"query {i} selection"
+
+
 # ------------------------------------------------------------------ A6 prefill chunk
 def test_prefill_chunk_matches_oracle():
     """A causal prefill chunk (the C4 shape, reduced): 96 queries at positions

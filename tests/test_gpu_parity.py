@@ -416,6 +416,17 @@ def test_plan_paged_ragged_batch():
     _check_plan(c)
 
 
+def test_plan_verify_block_of_five_queries():
+    """A speculative-verify block: 5 queries of one sequence at consecutive
+    positions, each with its own full / reindex / reuse step, through one
+    plan call."""
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(30000,), prefill=(5, 29995),
+                      modes=(synth.FULL, synth.REINDEX, synth.REUSE))
+    c = G.build(wl)
+    assert len(c.query_pos) == 5 and (c.seq_of_query == 0).all()
+    _check_plan(c)
+
+
 def test_plan_tiny_config():
     c = G.build(synth.C0_TINY)
     _check_plan(c)

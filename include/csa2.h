@@ -32,7 +32,10 @@
  * Conventions for every entry point
  *   - Every pointer is a DEVICE pointer unless it is marked "host".  The caller
  *     allocates and owns every buffer.  The library never allocates or frees
- *     memory, never synchronises, and keeps no mutable global state.  Calls
+ *     memory and never synchronises.  Apart from the fixed scratch array of
+ *     csa2_topk_pool_noalloc (see there), its only global state is one-time,
+ *     per-device set-up (kernel attributes, occupancy figures), held in
+ *     atomics, so first calls from several host threads do not race.  Calls
  *     that use distinct workspaces and streams are independent.
  *   - All work is enqueued on `stream` (a cudaStream_t; NULL means the legacy
  *     default stream).  Nothing is complete when the call returns.

@@ -476,13 +476,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};   // looked up again until found
+  EncodeTiledFn fn = cached.load(std::memory_order_acquire);
   if (!fn) {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult qr;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) == cudaSuccess &&
-        qr == cudaDriverEntryPointSuccess)
+        qr == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(p);
+      cached.store(fn, std::memory_order_release);
+    }
   }
   return fn;
 }
@@ -499,7 +502,7 @@ size_t index_smem_bytes(int N, int QG, int nq) {
 template <int D, int N, int QG>
 cudaError_t launch_one(const CUtensorMap& map, const IndexArgs& a, int grid, cudaStream_t st) {
   const size_t smem = index_smem_bytes<D>(N, QG, a.nq);
-  static unsigned long long done = 0;
+  static SetupMask done{0};
   cudaError_t e = ensure_smem(index_score_kernel<D, N, QG>, (int)index_smem_bytes<D>(N, QG, kMaxQueries), done);
   if (e != cudaSuccess) return e;
   return launch_k(index_score_kernel<D, N, QG>, dim3(grid), dim3(64 + kEpiThreads), smem, st, false,

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "csa2.h"
 
 namespace csa2 {
@@ -190,9 +192,14 @@ cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64
 
 int sm_count();
 
+// One-time, per-device set-up (a kernel's shared-memory limit, an occupancy
+// figure) is cached in atomics: host threads that make their first calls at
+// the same time at worst repeat the set-up, and never race.
+using SetupMask = std::atomic<unsigned long long>;   // bit d: done on device d
+
 // Raises a kernel's dynamic shared-memory limit once per device.
 template <class F>
-cudaError_t ensure_smem(F* kernel, int bytes, unsigned long long& done_mask) {
+cudaError_t ensure_smem(F* kernel, int bytes, SetupMask& done_mask) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;

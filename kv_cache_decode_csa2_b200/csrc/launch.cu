@@ -7,7 +7,9 @@ namespace csa2 {
 
 namespace {
 thread_local LaunchOpts t_opts;
-bool g_pdl_off = false;   // set once a programmatic launch was refused
+// Set when a launch with the programmatic-serialisation attribute failed and
+// the same launch without it succeeded: later launches leave it out.
+std::atomic<bool> g_pdl_off{false};
 }  // namespace
 
 LaunchOpts& launch_opts() { return t_opts; }
@@ -26,7 +28,7 @@ cudaError_t launch_ex(const void* kernel, void** args, dim3 grid, dim3 block, si
     attr[n].val.cooperative = 1;
     ++n;
   }
-  const bool use_pdl = pdl && !g_pdl_off;
+  const bool use_pdl = pdl && !g_pdl_off.load(std::memory_order_relaxed);
   if (use_pdl) {
     attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[n].val.programmaticStreamSerializationAllowed = 1;
@@ -35,11 +37,11 @@ cudaError_t launch_ex(const void* kernel, void** args, dim3 grid, dim3 block, si
   cfg.attrs = attr;
   cfg.numAttrs = n;
   cudaError_t e = cudaLaunchKernelExC(&cfg, kernel, args);
-  if (e != cudaSuccess && use_pdl) {
+  if (e != cudaSuccess && use_pdl) {   // retry without the programmatic attribute (the last one)
     (void)cudaGetLastError();
-    g_pdl_off = true;
     cfg.numAttrs = n - 1;
     e = cudaLaunchKernelExC(&cfg, kernel, args);
+    if (e == cudaSuccess) g_pdl_off.store(true, std::memory_order_relaxed);
   }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

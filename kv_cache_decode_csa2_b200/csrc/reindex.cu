@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(128) reindex_score_kernel(const ReindexArgs a)
 template <int D, int N>
 cudaError_t launch_r(const ReindexArgs& a, int nq, cudaStream_t st) {
   const size_t smem = 1024 + 128 * D + N * D + 128 * 4 + 64;
-  static unsigned long long done = 0;
+  static SetupMask done{0};
   cudaError_t e = ensure_smem(reindex_score_kernel<D, N>, (int)smem, done);
   if (e != cudaSuccess) return e;
   const dim3 grid((a.P + 127) / 128, nq);
@@ -448,8 +448,8 @@ template <int D, int N, int T>
 cudaError_t launch_rs_t(const RSelArgs& a_in, int n_jobs, int nq, size_t zero_bytes, cudaStream_t st) {
   using Lay = RSelLayout<D, N, T>;
   constexpr size_t smem = Lay::smem;
-  static unsigned long long done = 0;
-  static int max_ctas[64];
+  static SetupMask done{0};
+  static std::atomic<int> max_ctas[64];   // co-resident CTAs per device (0: not yet known)
   cudaError_t e = ensure_smem(reindex_select_kernel<D, N, T>, (int)smem, done);
   if (e != cudaSuccess) return e;
   int dev = 0;

@@ -474,8 +474,8 @@ __global__ void __launch_bounds__(NTHR) attn_merge_kernel(const __grid_constant_
 template <int D, int HG, int NTHR>
 cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
   using L = AttnSmem<D, HG>;
-  static unsigned long long done = 0;
-  static int max_ctas[64];
+  static SetupMask done{0};
+  static std::atomic<int> max_ctas[64];   // co-resident CTAs per device (0: not yet known)
   cudaError_t e = ensure_smem(sparse_attn_kernel<D, HG, NTHR>, (int)L::total, done);
   if (e != cudaSuccess) return e;
   int dev = 0;

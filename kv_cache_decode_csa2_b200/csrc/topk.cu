@@ -591,7 +591,7 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
   GatherArgs ga{v, s, n_k, status};
   topk_gather_kernel<<<grid, 256, 0, st>>>(ga);
   const int smem = (kCandCap + kTieCap) * 8;
-  static unsigned long long done = 0;
+  static SetupMask done{0};
   e = ensure_smem(topk_finish_kernel, smem, done);
   if (e != cudaSuccess) return e;
   FinishArgs fa{v, s, {outs[0], n_k > 1 ? outs[1] : outs[0]}};

@@ -20,7 +20,7 @@ constexpr size_t kNoallocScratchBytes = (size_t)CSA2_NOALLOC_SCRATCH_BYTES;
 // a device address: the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_topk_scratch[kNoallocScratchBytes];
 
-void* g_scratch_addr[64];   // device address of g_topk_scratch, per device id (set-up once)
+std::atomic<void*> g_scratch_addr[64];   // device address of g_topk_scratch, per device id (set-up once)
 
 // Looks up the array's address on the current device the first time the
 // entry point runs there.

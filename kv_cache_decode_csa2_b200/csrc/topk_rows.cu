@@ -409,7 +409,7 @@ cudaError_t launch_row_select(const int32_t* scores, int64_t ld, const int32_t* 
                               const int32_t* query_pos, const int32_t* cand_pos, int32_t nq, int32_t n_max,
                               const TopkOut* outs, int32_t n_k, int32_t* status, cudaStream_t st) {
   if (n_max > kRowSelMax || n_k < 1 || n_k > 2) return cudaErrorNotSupported;
-  static unsigned long long done1 = 0, done2 = 0;
+  static SetupMask done1{0}, done2{0};
   cudaError_t e = n_k == 1 ? ensure_smem(row_select_kernel<1>, kRowSmem, done1)
                            : ensure_smem(row_select_kernel<2>, kRowSmem, done2);
   if (e != cudaSuccess) return e;

@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
 }
 
 struct SelDev {
-  int max_ctas = 0;
+  std::atomic<int> max_ctas{0};   // co-resident CTAs of select_kernel<8> (0: not yet known)
 };
 SelDev g_sel_dev[64];
 
@@ -345,7 +345,7 @@ bool select_fits(int32_t nq, int32_t n_max) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
   SelDev& d = g_sel_dev[dev];
   if (!d.max_ctas) {
-    static unsigned long long done = 0;
+    static SetupMask done{0};
     int per_sm = 0;
     if (ensure_smem(select_kernel<8>, kSelSmem, done) != cudaSuccess ||
         cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, select_kernel<8>, kSelNT, kSelSmem) != cudaSuccess)
@@ -370,7 +370,7 @@ cudaError_t launch_select(const int32_t* scores, int64_t ld, const int32_t* n_va
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  static unsigned long long done16 = 0, done8 = 0;
+  static SetupMask done16{0}, done8{0};
   e = one ? ensure_smem(select_kernel<16>, kSelSmem, done16) : ensure_smem(select_kernel<8>, kSelSmem, done8);
   if (e != cudaSuccess) return e;
   if (G > 1) {

@@ -294,6 +294,28 @@ int32_t csa2_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_
 const char* csa2_status_string(int32_t status);  /* static string, never NULL */
 int32_t csa2_version(void);                       /* major*10000 + minor*100 + patch */
 
+/* ------------------------------------------------------------ phase tracing
+ * In the traced build of the library (libcsa2_trace.so, compiled with
+ * -DCSA2_TRACE) the kernels carry phase markers: one thread of every CTA
+ * records two uint64 values at each marked point of its kernel, the global
+ * timer (ns) and the SM clock cycles since it entered the kernel.
+ *   csa2_trace_table_bytes  size of the table: uint64
+ *                           [8 kernels][1024 CTAs][16 points][2]; kernels are
+ *                           0 index score, 1 select, 2 fused reindex,
+ *                           3 attention, 4 row select, 5 zeroing; point 0 is
+ *                           kernel entry.  CTA = x + X*(y + Y*z) of its grid;
+ *                           CTAs past 1024 are not recorded.
+ *   csa2_trace_attach       table: device memory of that size (8-byte aligned),
+ *                           zeroed by the caller, or NULL to stop recording.
+ *                           It applies to the current device.  Points a
+ *                           kernel did not reach stay zero, and each launch
+ *                           overwrites the entries of the one before.
+ * The normal build compiles the markers to nothing; there csa2_trace_attach
+ * returns CSA2_ERR_UNSUPPORTED and touches nothing.
+ */
+size_t csa2_trace_table_bytes(void);
+int32_t csa2_trace_attach(void* table);
+
 #ifdef __cplusplus
 }
 #endif

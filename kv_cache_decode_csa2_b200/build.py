@@ -1,8 +1,11 @@
 """Builds libcsa2.so in-tree from csrc/*.cu for sm_100a (B200) with nvcc.
 
-Usage: python -m kv_cache_decode_csa2_b200.build   (or build() from Python).
+Usage: python -m kv_cache_decode_csa2_b200.build [--trace]   (or build()).
 Objects go to csrc/_build/; a source is recompiled when it or any header is
-newer than its object.
+newer than its object.  With --trace (build(trace=True)) the same sources are
+compiled with -DCSA2_TRACE, which turns the kernels' phase markers on, into
+libcsa2_trace.so (objects in csrc/_build_trace/); see csa2_trace_attach in
+include/csa2.h.
 """
 from __future__ import annotations
 
@@ -17,6 +20,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(CSRC, "_build")
 LIB = os.path.join(HERE, "libcsa2.so")
+OBJ_TRACE = os.path.join(CSRC, "_build_trace")
+LIB_TRACE = os.path.join(HERE, "libcsa2_trace.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-Wall",
@@ -36,18 +41,20 @@ def _newest_header() -> float:
     return max(os.path.getmtime(h) for h in hdrs)
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+def build(verbose: bool = False, force: bool = False, trace: bool = False) -> str:
+    obj_dir, lib = (OBJ_TRACE, LIB_TRACE) if trace else (OBJ, LIB)
+    flags = FLAGS + (["-DCSA2_TRACE"] if trace else [])
+    os.makedirs(obj_dir, exist_ok=True)
     nvcc = _nvcc()
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_t = _newest_header()
     jobs = []
     objs = []
     for src in srcs:
-        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(obj_dir, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr_t):
-            jobs.append([nvcc, *ARCH, *FLAGS, "-c", src, "-o", obj])
+            jobs.append([nvcc, *ARCH, *flags, "-c", src, "-o", obj])
 
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -58,10 +65,11 @@ def build(verbose: bool = False, force: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(max(1, min(8, os.cpu_count() or 1))) as ex:
         list(ex.map(run, jobs))
-    if jobs or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        run([nvcc, *ARCH, "-shared", "-o", LIB, *objs])
-    return LIB
+    if jobs or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        run([nvcc, *ARCH, "-shared", "-o", lib, *objs])
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose=True))
+    import sys
+    print(build(verbose=True, trace="--trace" in sys.argv[1:]))

@@ -76,6 +76,8 @@ _SIGS = {
     "csa2_fp4_quantize": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
     "csa2_status_string": (ctypes.c_char_p, [_I32]),
     "csa2_version": (_I32, []),
+    "csa2_trace_table_bytes": (_SZ, []),
+    "csa2_trace_attach": (_I32, [_P]),
 }
 EXPORTS = tuple(_SIGS)
 

@@ -105,6 +105,25 @@ const char* csa2_status_string(int32_t s) {
 
 int32_t csa2_version(void) { return 100; }   // 0.1.0
 
+size_t csa2_trace_table_bytes(void) {
+  return (size_t)kTraceKernels * kTraceCtas * kTracePhases * 2 * sizeof(uint64_t);
+}
+
+int32_t csa2_trace_attach(void* table) {
+#ifdef CSA2_TRACE
+  if (table && !aligned(table, 8)) return CSA2_ERR_INVALID_ARG;
+  uint64_t* t = static_cast<uint64_t*>(table);
+  cudaError_t (*const attach[])(uint64_t*) = {trace_attach_index, trace_attach_select, trace_attach_reindex,
+                                               trace_attach_attn,  trace_attach_rows,   trace_attach_zero};
+  for (auto f : attach)
+    if (f(t) != cudaSuccess) return CSA2_ERR_CUDA;
+  return CSA2_OK;
+#else
+  (void)table;
+  return CSA2_ERR_UNSUPPORTED;   // phase markers are compiled in only in the traced build
+#endif
+}
+
 size_t csa2_index_full_workspace(int32_t nq, int32_t max_ctx, int32_t P, int32_t K) {
   if (nq < 1 || max_ctx < 1) return 0;
   return index_full_ws(nq, max_ctx, P, K, nullptr, nullptr, nullptr);

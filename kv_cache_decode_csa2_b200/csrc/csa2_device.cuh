@@ -31,6 +31,53 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// ------------------------------------------------------------------ tracing
+// Phase markers.  The normal build compiles them to nothing.  The traced build
+// (-DCSA2_TRACE, libcsa2_trace.so) has one chosen thread of every CTA record
+// two values at each marked point: the global timer, and the SM cycles since
+// the thread entered the kernel.  They go into a caller-owned table attached
+// with csa2_trace_attach(): uint64 [kTraceKernels][kTraceCtas][kTracePhases][2].
+// Entries stay zero for points that were not reached, and CTAs past
+// kTraceCtas are not recorded.  A later launch of the same kernel overwrites
+// the entries of an earlier one.
+constexpr int kTraceKernels = 8;
+constexpr int kTraceCtas = 1024;
+constexpr int kTracePhases = 16;
+enum TraceKernel : int { kTrIndex = 0, kTrSelect = 1, kTrReindex = 2, kTrAttn = 3, kTrRowSel = 4, kTrZero = 5 };
+#ifdef CSA2_TRACE
+__device__ __forceinline__ void trace_mark(uint64_t* table, int kernel, int phase, long long t0) {
+  const uint32_t cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+  if (!table || cta >= (uint32_t)kTraceCtas || (uint32_t)phase >= (uint32_t)kTracePhases ||
+      (uint32_t)kernel >= (uint32_t)kTraceKernels)
+    return;
+  uint64_t* e = table + (((size_t)kernel * kTraceCtas + cta) * kTracePhases + phase) * 2;
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  e[0] = t;
+  e[1] = (uint64_t)(clock64() - t0);
+}
+// Once per translation unit with markers, at namespace csa2 scope before its
+// kernels: the unit's table pointer and the host function that sets it.
+#define CSA2_TRACE_UNIT(name)                               \
+  static __device__ uint64_t* trace_table_ = nullptr;       \
+  cudaError_t trace_attach_##name(uint64_t* p) {            \
+    return cudaMemcpyToSymbol(trace_table_, &p, sizeof(p)); \
+  }
+// At the top of a kernel (phase 0), then at each marked point; `who` picks the
+// recording thread.
+#define CSA2_TRACE_BEGIN(kernel, who)        \
+  const long long trace_t0_ = clock64();     \
+  if (who) trace_mark(trace_table_, kernel, 0, trace_t0_)
+#define CSA2_MARK(kernel, phase, who)                                   \
+  do {                                                                  \
+    if (who) trace_mark(trace_table_, kernel, phase, trace_t0_);        \
+  } while (0)
+#else
+#define CSA2_TRACE_UNIT(name)
+#define CSA2_TRACE_BEGIN(kernel, who) ((void)0)
+#define CSA2_MARK(kernel, phase, who) ((void)0)
+#endif
+
 // Programmatic dependent launch.  pdl_wait() blocks until the grid this one
 // depends on has completed and its writes are visible (a no-op when the
 // launch has no such dependency); pdl_trigger() lets the next grid of the

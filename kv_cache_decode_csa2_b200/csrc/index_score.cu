@@ -25,6 +25,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(index)
+
 namespace {
 
 struct IndexArgs {
@@ -99,6 +101,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
+  // trace points: 1 prologue done, 2 first TMA issued, 3 first stage landed,
+  // 4 first epilogue tile done, 5 last epilogue tile done, 6 histogram
+  // flushed, 7 producer done, 8 MMA issuer done, 9 exit
+  CSA2_TRACE_BEGIN(kTrIndex, tid == 0);
 
   // ---- prologue: warp 0 builds the work list (groups of queries and the
   // tiles before each group), warp 1 allocates TMEM, thread 0 sets up the
@@ -187,6 +193,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int ngroups = *ngroups_s;
+  CSA2_MARK(kTrIndex, 1, tid == 0);
   pdl_trigger();   // the next grid may be launched (it waits for this one to finish)
   if (warp >= 2) {   // the epilogue's histogram, zeroed before its first use
     for (int i = tid - 64; i < kHist; i += kEpiThreads) hist_s[i] = 0;
@@ -300,6 +307,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           for (int j = 0; j < 2; ++j)
             if (r[j] >= 0)
               tma_load_2d(stages + st * TILE + j * 64 * D, &kmap, 0, (int32_t)r[j], &full[st], pol);
+          CSA2_MARK(kTrIndex, 2, gi == 0);
         }
         if (*abort_flag) {   // let loads already in flight land before moving on
           const int64_t issued = git + i;
@@ -307,6 +315,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           for (int64_t k = issued - n; k < issued; ++k)
             mbar_wait_drain(&full[k % NST], (uint32_t)((k / NST) & 1));
         }
+        CSA2_MARK(kTrIndex, 7, true);
       }
     } else if (warp == 1) {
       // ---------------------------------------------------------- MMA issuer
@@ -322,6 +331,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           const int buf = (int)(gi % NBUF);
           const uint32_t tph = (uint32_t)((gi / NBUF) & 1);
           if (!mbar_wait(&full[st], ph, abort_flag)) break;
+          CSA2_MARK(kTrIndex, 3, gi == 0);
           if (!mbar_wait(&tempty[buf], tph ^ 1, abort_flag)) break;
           tc_fence_after();
           const uint32_t a_addr = smem_u32(stages + st * TILE);
@@ -332,6 +342,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           mma_commit(&empty[st]);
           mma_commit(&tfull[buf]);
         }
+        CSA2_MARK(kTrIndex, 8, true);
       }
     } else {
       // ---------------------------------------------------------- epilogue
@@ -436,7 +447,9 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
         }
+        CSA2_MARK(kTrIndex, 4, tid == 64 && gi == 0);
       }
+      CSA2_MARK(kTrIndex, 5, tid == 64);
       // this query's histogram goes to global memory
       named_sync_epi();
       if constexpr (QG == 1) {
@@ -450,6 +463,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           }
         }
       }
+      CSA2_MARK(kTrIndex, 6, tid == 64);
     }
     tc_fence_before();
     __syncthreads();   // the segment is done everywhere: B and the histogram may be reused
@@ -466,6 +480,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     s_lo = s_hi;
   }
 
+  CSA2_MARK(kTrIndex, 9, tid == 0);
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
   if (tid == 0 && *abort_flag) record_error(a.status, CSA2_ERR_TIMEOUT);
 }

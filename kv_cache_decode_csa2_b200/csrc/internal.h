@@ -192,6 +192,16 @@ cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64
 
 int sm_count();
 
+#ifdef CSA2_TRACE
+// The traced build: each translation unit with phase markers sets its table.
+cudaError_t trace_attach_index(uint64_t* table);
+cudaError_t trace_attach_select(uint64_t* table);
+cudaError_t trace_attach_reindex(uint64_t* table);
+cudaError_t trace_attach_attn(uint64_t* table);
+cudaError_t trace_attach_rows(uint64_t* table);
+cudaError_t trace_attach_zero(uint64_t* table);
+#endif
+
 // One-time, per-device set-up (a kernel's shared-memory limit, an occupancy
 // figure) is cached in atomics: host threads that make their first calls at
 // the same time at worst repeat the set-up, and never race.

@@ -5,6 +5,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(zero)
+
 namespace {
 thread_local LaunchOpts t_opts;
 // Set when a launch with the programmatic-serialisation attribute failed and
@@ -54,8 +56,10 @@ struct ZeroArgs {
   int32_t n;
 };
 __global__ void __launch_bounds__(256) zero_kernel(const __grid_constant__ ZeroArgs a) {
+  CSA2_TRACE_BEGIN(kTrZero, threadIdx.x == 0);   // trace point 1: done
   for (int r = 0; r < a.n; ++r)
     for (uint32_t i = blockIdx.x * 256 + threadIdx.x; i < a.words[r]; i += gridDim.x * 256) a.ptr[r][i] = 0u;
+  CSA2_MARK(kTrZero, 1, threadIdx.x == 0);
 }
 }  // namespace
 

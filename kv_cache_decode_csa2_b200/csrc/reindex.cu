@@ -23,6 +23,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(reindex)
+
 namespace {
 
 struct ReindexArgs {
@@ -226,6 +228,10 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   const RSelJob& J = a.job[jb];
   const int prob = jb * a.nq + q;
   const int G = a.G;
+  // trace points: 1 own inputs staged, 2 grid before done, 3 pool rows
+  // gathered, 4 scored, 5 histogram barrier, 6 threshold bucket, 7 tie
+  // barrier, 8 ties ranked, 9 count barrier, 10 written
+  CSA2_TRACE_BEGIN(kTrReindex, tid == 0);
   if (tid == 0) {
     bstar_s = -1;
     above_s = 0;
@@ -253,8 +259,10 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     }
     if (tid < N) w_s[tid] = tid < a.H ? (int32_t)__ldg(J.w + (int64_t)q * a.H + tid) : 0;
   }
+  CSA2_MARK(kTrReindex, 1, tid == 0);
   pdl_wait();      // the pool comes from the grid before
   pdl_trigger();
+  CSA2_MARK(kTrReindex, 2, tid == 0);
 
   int32_t cnt = __ldg(a.pool_cnt + q);
   cnt = cnt < 0 ? 0 : (cnt > a.P ? a.P : cnt);
@@ -291,6 +299,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  CSA2_MARK(kTrReindex, 3, tid == 0);
   const uint32_t tmem_base = *tmem_slot;
   if (has) {
     if (tid == 0) {
@@ -332,6 +341,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   }
   tc_fence_before();
   __syncthreads();   // also: the tiles are free for the tie list from here on
+  CSA2_MARK(kTrReindex, 4, tid == 0);
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
@@ -345,6 +355,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   if (valid) atomicAdd(&hist[bk], 1u);
   uint32_t phase = 0;
   sel_grid_sync(&hdr[0], ++phase * G, a.status);
+  CSA2_MARK(kTrReindex, 5, tid == 0);
   constexpr int kBins = kBuckets / NT;   // bins per thread
   uint4 hv[kBins / 4];
   const uint4* hp = reinterpret_cast<const uint4*>(hist + tid * kBins);
@@ -376,6 +387,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     }
   }
   __syncthreads();
+  CSA2_MARK(kTrReindex, 6, tid == 0);
   const int32_t bstar = bstar_s;   // -1: every valid entry is a member
 
   // ---- ties at b*: ranked against the pool's tie list
@@ -389,6 +401,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
       if (g < (uint32_t)kRTieCap) a.ties[(size_t)prob * kRTieCap + g] = key;
     }
     sel_grid_sync(&hdr[0], ++phase * G, a.status);
+    CSA2_MARK(kTrReindex, 7, tid == 0);
     const uint32_t nt = __ldcg(&hdr[1]);
     const int32_t need = K - above_s;
     if (nt <= (uint32_t)kRTieCap) {
@@ -411,6 +424,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
       if (tid == 0) kthr_s = kth;
     }
     __syncthreads();
+    CSA2_MARK(kTrReindex, 8, tid == 0);
   }
   const bool member = above || (tie && key >= kthr_s);
 
@@ -427,6 +441,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   uint32_t* mc = a.mcnt + (size_t)prob * G;
   if (tid == 0) mc[x] = cta_cnt;
   sel_grid_sync(&hdr[0], ++phase * G, a.status);
+  CSA2_MARK(kTrReindex, 9, tid == 0);
   uint64_t part = 0ull;   // (members of the CTAs before) | (all members) << 32
   for (int r = tid; r < G; r += NT) {
     const uint64_t v = __ldcg(mc + r);
@@ -442,6 +457,7 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     for (int32_t i = n_out + tid; i < K; i += NT) dst[i] = -1;
     if (tid == 0 && J.sel_cnt) J.sel_cnt[q] = n_out;
   }
+  CSA2_MARK(kTrReindex, 10, tid == 0);
 }
 
 template <int D, int N, int T>

@@ -30,6 +30,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(attn)
+
 namespace {
 
 constexpr int kCl = 8;       // CTAs per group: row slices of one (layer, query, head group)
@@ -230,6 +232,10 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
   const int job_i = blockIdx.z / a.nq, q = blockIdx.z % a.nq;
   const AttnJob& J = a.jobs[job_i];
   const int h0 = hg * HG;
+  // trace points: 1 Q staged, 2 grid before done, 3 row positions, 4 rows
+  // gathered and dequantised, 5 logits, 6 softmax, 7 P V done, 8 partial
+  // written, 9 group barrier, 10 merged (3-6: the last tile)
+  CSA2_TRACE_BEGIN(kTrAttn, tid == 0);
 
   // ---- independent loads first: Q rows of this head group, position, count
   constexpr int QPER = HG * (D / 8) / NTHR;
@@ -252,8 +258,10 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
     ml_s[tid * 4 + 0] = -INFINITY;
     ml_s[tid * 4 + 1] = 0.f;
   }
+  CSA2_MARK(kTrAttn, 1, tid == 0);
   pdl_wait();      // the selection comes from the grid before
   pdl_trigger();
+  CSA2_MARK(kTrAttn, 2, tid == 0);
   int32_t cnt = J.sel_cnt ? __ldg(J.sel_cnt + q) : a.K;
   if (tid == 0 && rank == 0 && pos < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
 
@@ -308,6 +316,7 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
       row_s[kTile + tid] = sr;
     }
     __syncthreads();
+    CSA2_MARK(kTrAttn, 3, tid == 0);
     // ---- gather + dequantise: one (row, 8-element group) per item, so a warp
     // reads 128 consecutive code bytes of a row and writes 512 consecutive
     // bytes of shared memory.  All loads of a thread are issued before any use.
@@ -332,6 +341,7 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
       }
     }
     __syncthreads();
+    CSA2_MARK(kTrAttn, 4, tid == 0);
     // ---- logits: S[h][r] = Q[h] . KV[r]
     {
       // with registers to spare, two accumulators per n-tile (even and odd k)
@@ -378,6 +388,7 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
       }
     }
     __syncthreads();
+    CSA2_MARK(kTrAttn, 5, tid == 0);
     // ---- online softmax: TPH threads per head, RPT rows each
     {
       const int h = tid / TPH, part = tid % TPH;
@@ -412,6 +423,7 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
       }
     }
     __syncthreads();
+    CSA2_MARK(kTrAttn, 6, tid == 0);
     // ---- O[h][d] = alpha[h] O[h][d] + sum_r P[h][r] KV[r][d]
     {
       const int d0 = wj * DW, g = lane >> 2;
@@ -441,6 +453,7 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
     }
     // the next tile's position pass ends with a barrier before the K/V tile is rewritten
   }
+  CSA2_MARK(kTrAttn, 7, tid == 0);
 
   // ---- this CTA's partial (max, sum, O) to L2, then the merge of the group
   {
@@ -455,9 +468,12 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
     }
     if (tid < HG) a.part_ml[((size_t)gidx * kCl + rank) * HG + tid] = make_float2(ml_s[tid * 4], ml_s[tid * 4 + 1]);
   }
+  CSA2_MARK(kTrAttn, 8, tid == 0);
   if (!a.fused) return;
   sel_grid_sync(a.bar + gidx, kCl, a.status);
+  CSA2_MARK(kTrAttn, 9, tid == 0);
   merge_slice<D, HG, NTHR>(a, J, q, h0, gidx, rank, s_s);
+  CSA2_MARK(kTrAttn, 10, tid == 0);
 }
 
 // The merge of every group, when the attention CTAs could not all be resident.

@@ -24,6 +24,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(rows)
+
 namespace {
 
 constexpr int kRowNT = 1024;
@@ -73,6 +75,9 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = blockIdx.x;
   constexpr int n_k = NK;
+  // trace points: 1 threshold buckets, 2 score bounds, 3 classified, 4 ties
+  // resolved, 5 written
+  CSA2_TRACE_BEGIN(kTrRowSel, tid == 0);
   const int32_t n = row_n(a, q);
   const int32_t R = (((n + kRowNT - 1) / kRowNT) + 3) & ~3;   // candidates per thread, a multiple of 4
   const int32_t j0 = tid * R;
@@ -226,6 +231,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     __syncthreads();
   }
   __syncthreads();
+  CSA2_MARK(kTrRowSel, 1, tid == 0);
 
   // ---- pass 2: members above b* and ties at b*, as bitmasks
   const int32_t b0 = bstar_s[0], b1 = n_k > 1 ? bstar_s[1] : INT32_MIN;
@@ -239,6 +245,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     bound_s[tid] = (t >= n_k || bs < 0) ? 0ll : b >= kBuckets ? (long long)INT32_MAX + 1 : bucket_min_score(b);
   }
   __syncthreads();
+  CSA2_MARK(kTrRowSel, 2, tid == 0);
   const long long lo0 = bound_s[0], hi0 = bound_s[1], lo1 = bound_s[2], hi1 = bound_s[3];
   const bool all0 = b0 < 0, all1 = n_k > 1 && b1 < 0;
   uint32_t above_m[NK][kRowWords], tie_m[NK][kRowWords];
@@ -286,6 +293,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     }
   }
   __syncthreads();
+  CSA2_MARK(kTrRowSel, 3, tid == 0);
   // rank the ties: the members among them are those with fewer than need
   // better ties; the smallest such key is the threshold key
 #pragma unroll
@@ -357,6 +365,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     if (tid == 0) kthr_s[t] = prefix;
   }
   __syncthreads();
+  CSA2_MARK(kTrRowSel, 4, tid == 0);
 
   // ---- members: ties at or above the threshold key join the bitmasks
   const uint64_t kthr[2] = {kthr_s[0], kthr_s[1]};
@@ -399,6 +408,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     for (int32_t i = c + tid; i < k; i += kRowNT) dst[i] = -1;
     if (tid == 0 && a.out_cnt[t]) a.out_cnt[t][q] = c;
   }
+  CSA2_MARK(kTrRowSel, 5, tid == 0);
 }
 
 constexpr int kRowSmem = kBuckets * 4 + 2 * kRowTieCap * 8;

@@ -30,6 +30,8 @@
 
 namespace csa2 {
 
+CSA2_TRACE_UNIT(select)
+
 namespace {
 
 constexpr int kBinsPer = kBuckets / kSelNT;
@@ -92,6 +94,10 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int q = blockIdx.y, c = blockIdx.x, G = a.G, n_k = a.n_k;
   const int32_t j0 = c * kSpan + tid * E;
+  // trace points: 1 grid before done, 2 threshold buckets, 3 classified,
+  // 4 first grid barrier, 5 row ties staged, 6 ties ranked, 7 second grid
+  // barrier, 8 written
+  CSA2_TRACE_BEGIN(kTrSelect, tid == 0);
   const int32_t* row = a.scores + (int64_t)q * a.ld;
   uint32_t phase = 0;   // grid barriers passed
   uint32_t* hdr = a.hdr ? a.hdr + q * 4 : nullptr;
@@ -103,6 +109,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
   }
   pdl_wait();      // the scores, the histogram and the counts come from the grid before
   pdl_trigger();
+  CSA2_MARK(kTrSelect, 1, tid == 0);
   const int32_t n = sel_n(a, q);
 
   // ---- 1. loads: scores (up to n_max, which the row always holds; masked by
@@ -184,6 +191,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
     }
   }
   __syncthreads();
+  CSA2_MARK(kTrSelect, 2, tid == 0);
 
   // ---- 3. classify: above b* (members), at b* (ties: this CTA's list)
   const int32_t b0 = bstar_s[0], b1 = n_k > 1 ? bstar_s[1] : INT32_MIN;
@@ -208,6 +216,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
     }
   }
   __syncthreads();
+  CSA2_MARK(kTrSelect, 3, tid == 0);
   const uint32_t* nt = own_cnt;   // ties in the row
   const uint64_t* list = own;     // the row's ties, [2][kSelTieCap]
   if (G > 1) {
@@ -221,6 +230,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
         if (gbase_s[t] + i < (uint32_t)kSelTieCap) dst[gbase_s[t] + i] = own[t * kSelTieCap + i];
     }
     sel_grid_sync(&hdr[0], ++phase * G, a.status);
+    CSA2_MARK(kTrSelect, 4, tid == 0);
     if (tid < 2) nt_s[tid] = __ldcg(&hdr[1 + tid]);
     __syncthreads();
 #pragma unroll
@@ -234,6 +244,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
     nt = nt_s;
     list = rowties;
     __syncthreads();
+    CSA2_MARK(kTrSelect, 5, tid == 0);
   }
   // rank this CTA's ties against the row's ties
 #pragma unroll
@@ -262,6 +273,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
     if (tid == 0) kthr_s[t] = kth;
   }
   __syncthreads();
+  CSA2_MARK(kTrSelect, 6, tid == 0);
 
   // ---- 4. members, their slots and the ordered write
   uint32_t mem[2] = {above_m[0], above_m[1]};
@@ -286,6 +298,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
       mc[kSelMaxG + c] = (uint32_t)(cta_tot >> 32);
     }
     sel_grid_sync(&hdr[0], ++phase * G, a.status);
+    CSA2_MARK(kTrSelect, 7, tid == 0);
     if (warp == 0) {
       uint64_t o = 0ull, g = 0ull;
       for (int r = lane; r < G; r += 32) {
@@ -328,6 +341,7 @@ __global__ void __launch_bounds__(kSelNT, 1) select_kernel(const __grid_constant
       if (tid == 0 && a.out_cnt[t]) a.out_cnt[t][q] = cnt;
     }
   }
+  CSA2_MARK(kTrSelect, 8, tid == 0);
 }
 
 struct SelDev {

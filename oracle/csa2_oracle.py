@@ -45,6 +45,10 @@ see tests/test_oracle_pins.py):
                       the set is the whole context; closed forms.
   decode_layer_plan   pinned: separate pure-Python brute force on tiny inputs.
   prefill_query       pinned: equals decode at the same position (property).
+  kv_rows_local_window  pinned: closed forms (one window row, uniform
+                      softmax over ring slots and FP4 rows), the separate
+                      brute force of the plan with local rings, and equality
+                      with the FP4-only rows when the ring holds them.
 """
 from __future__ import annotations
 
@@ -286,6 +290,39 @@ def sparse_attention(q: np.ndarray, kv_rows: np.ndarray, softmax_scale: float | 
     return o, (mx + np.log(l))[:, 0]
 
 
+# =============================================================== the layer's local window cache
+def kv_rows_local_window(S, pos: int, window: int, codes, scales, D: int, local_ring) -> np.ndarray:
+    """Key/value rows of the attention set S (ascending positions, as
+    attention_set gives it) for a layer that keeps its own cache of the most
+    recent tokens beside the FP4 main cache.
+
+    The positions of the window [max(0, pos-window+1), pos] are read from
+    ``local_ring``, float [R][D] with R >= window: position p sits in slot
+    p mod R.  Every other position of S is read from the FP4 main cache
+    (codes, scales) and dequantised.  Returns float64 [len(S)][D].
+
+    [YS] "The three KV-cache optimizations", item 3: besides the global KV,
+    V4 kept a separate per-layer local KV for the latest 128 tokens, and
+    V4.1 keeps that local cache while a session is active.
+    READING 15: the pages give the local cache no number format and state FP4
+    for the global KV only, so the local cache holds the rows as they are
+    (bf16 values in the library), in a ring of R rows per sequence.
+    """
+    S = np.asarray(S, dtype=np.int64)
+    ring = np.asarray(local_ring, dtype=np.float64)
+    R = ring.shape[0]
+    if R < window:
+        raise ValueError(f"local ring of {R} rows cannot hold a window of {window}")
+    wstart = max(0, pos - window + 1)
+    rows = np.empty((len(S), D), dtype=np.float64)
+    local = S >= wstart
+    far = S[~local]
+    if far.size:
+        rows[~local] = fp4_dequant(np.asarray(codes)[far], np.asarray(scales)[far], D)
+    rows[local] = ring[S[local] % R]
+    return rows
+
+
 # =============================================================== the layer plan
 @dataclass
 class LayerResult:
@@ -306,7 +343,10 @@ def decode_layer_plan(modes, layers, pos: int, pool: int, topk: int, window: int
       'q', 'w', 'keys'    int8 indexer query, head weights and key rows
                           (needed by FULL and REINDEX layers),
       'q_attn'            float [Hq][D] query (bf16 values),
-      'codes', 'scales'   the FP4 cache planes of that layer.
+      'codes', 'scales'   the FP4 cache planes of that layer,
+      'local_ring'        optional float [R][D]: the layer's local cache of
+                          the most recent tokens; the window reads it (see
+                          kv_rows_local_window).
     Modes: FULL scores every position and builds the pool.  REINDEX re-scores
     the most recent FULL layer's pool.  REUSE takes the selection of the most
     recent FULL or REINDEX layer unchanged.
@@ -332,7 +372,10 @@ def decode_layer_plan(modes, layers, pos: int, pool: int, topk: int, window: int
             raise ValueError(f"unknown mode {mode}")
         S = attention_set(sel, pos, window)
         D = np.asarray(L["q_attn"]).shape[1]
-        kv = fp4_dequant(L["codes"][S], L["scales"][S], D)
+        if L.get("local_ring") is not None:
+            kv = kv_rows_local_window(S, pos, window, L["codes"], L["scales"], D, L["local_ring"])
+        else:
+            kv = fp4_dequant(L["codes"][S], L["scales"][S], D)
         o, lse = sparse_attention(L["q_attn"], kv, softmax_scale)
         results.append(LayerResult(mode, layer_pool, sel, S, o, lse, scores))
     return results

@@ -81,8 +81,15 @@ def decode_step(modes, layers, pos, pool, topk, window):
         elif mode == 1:
             sc = {p: score(L["q"], L["w"], L["keys"][p]) for p in pool_set}
             sel = select(sc, topk)
-        S = sorted(set(sel) | set(range(max(0, pos - window + 1), pos + 1)))
+        wstart = max(0, pos - window + 1)
+        S = sorted(set(sel) | set(range(wstart, pos + 1)))
         D = len(L["q_attn"][0])
-        rows = [dequant_row(L["codes"][p], L["scales"][p], D) for p in S]
+        ring = L.get("local_ring")
+        rows = []
+        for p in S:
+            if ring is not None and p >= wstart:   # the layer's local cache: slot p mod ring length
+                rows.append([float(x) for x in ring[p % len(ring)]])
+            else:
+                rows.append(dequant_row(L["codes"][p], L["scales"][p], D))
         res.append((list(sel), S, attend(L["q_attn"], rows, 1.0 / math.sqrt(D))))
     return res

@@ -343,6 +343,82 @@ def test_prefill_query_equals_single_full_layer_decode():
         assert np.array_equal(o, r.out)
 
 
+# ------------------------------------------------------------------ the layer's local window cache
+def test_local_window_single_row_is_the_output():
+    rng = np.random.default_rng(11)
+    D, R = 32, 128
+    ring = rng.standard_normal((R, D))
+    codes = np.zeros((4, D // 2), np.uint8)
+    scales = np.zeros((4, D // 32), np.uint8)
+    S = O.attention_set(np.zeros(0, np.int64), 0, 128)          # pos 0: the window is position 0 alone
+    rows = O.kv_rows_local_window(S, 0, 128, codes, scales, D, ring)
+    assert np.array_equal(rows, ring[:1])
+    o, _ = O.sparse_attention(rng.standard_normal((3, D)), rows)
+    assert np.allclose(o, np.broadcast_to(ring[0], (3, D)), atol=1e-15)
+
+
+def test_local_window_uniform_softmax_closed_form():
+    # FP4 rows of exactly 1.0 (code 2 = 1.0 in both nibbles, E4M3 0x38 = 1.0);
+    # ring slot k holds the constant k + 1; q = 0 makes the softmax uniform,
+    # so the output is the plain mean of the rows of S.
+    D, R, window, pos = 64, 8, 5, 20
+    codes = np.full((pos + 1, D // 2), 0x22, np.uint8)
+    scales = np.full((pos + 1, D // 32), 0x38, np.uint8)
+    ring = np.repeat(np.arange(1, R + 1, dtype=np.float64)[:, None], D, axis=1)
+    sel = np.array([2, 7, 17])                                   # 17 lies in the window 16..20
+    S = O.attention_set(sel, pos, window)
+    assert S.tolist() == [2, 7, 16, 17, 18, 19, 20]
+    rows = O.kv_rows_local_window(S, pos, window, codes, scales, D, ring)
+    want = (1.0 + 1.0 + sum((p % R) + 1 for p in range(16, 21))) / 7
+    o, _ = O.sparse_attention(np.zeros((2, D)), rows)
+    assert np.allclose(o, want, atol=1e-14)
+    assert rows[0].tolist() == [1.0] * D and rows[-1].tolist() == [float(20 % R + 1)] * D
+
+
+def test_local_window_holding_the_fp4_rows_changes_nothing():
+    rng = np.random.default_rng(12)
+    modes = [0, 1, 2]
+    ctx, window, R = 200, 16, 24
+    layers = _tiny_layers(rng, len(modes), ctx, H=3, Di=8, Hq=2, D=64)
+    pos = ctx - 1
+    plain = O.decode_layer_plan(modes, layers, pos, 40, 8, window)
+    for L in layers:
+        ring = np.zeros((R, 64))
+        for p in range(ctx - R, ctx):
+            ring[p % R] = O.fp4_dequant(L["codes"][p:p + 1], L["scales"][p:p + 1], 64)[0]
+        L["local_ring"] = ring
+    local = O.decode_layer_plan(modes, layers, pos, 40, 8, window)
+    for a, b in zip(plain, local):
+        assert np.array_equal(a.attn_set, b.attn_set)
+        assert np.array_equal(a.out, b.out) and np.array_equal(a.lse, b.lse)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_plan_with_local_rings_matches_bruteforce(seed):
+    rng = np.random.default_rng(200 + seed)
+    ctx = int(rng.integers(1, 64))
+    modes = [0, 2, 1, 2]
+    window, R = 6, 9
+    layers = _tiny_layers(rng, len(modes), ctx, H=3, Di=4, Hq=2, D=64)
+    for i in (0, 2, 3):                                          # layer 1 keeps reading the FP4 cache
+        layers[i]["local_ring"] = rng.standard_normal((R, 64))
+    pos, pool, topk = ctx - 1, 12, 5
+    got = O.decode_layer_plan(modes, layers, pos, pool, topk, window)
+    bl = [dict(L, codes=L["codes"].tolist(), scales=L["scales"].tolist(), q_attn=L["q_attn"].tolist(),
+               keys=L["keys"].tolist(),
+               local_ring=None if L.get("local_ring") is None else L["local_ring"].tolist()) for L in layers]
+    want = BF.decode_step(modes, bl, pos, pool, topk, window)
+    for g, (sel, S, out) in zip(got, want):
+        assert g.sel_idx.tolist() == sel and g.attn_set.tolist() == S
+        assert np.allclose(g.out, np.array(out), rtol=1e-12, atol=1e-12)
+
+
+def test_local_window_needs_a_ring_as_long_as_the_window():
+    with pytest.raises(ValueError):
+        O.kv_rows_local_window(np.array([5]), 5, 8, np.zeros((6, 16), np.uint8), np.zeros((6, 1), np.uint8), 32,
+                               np.zeros((7, 32)))
+
+
 def test_plan_rejects_bad_first_mode():
     with pytest.raises(ValueError):
         O.decode_layer_plan([1, 0], [{}, {}], 0, 4, 2, 2)

@@ -233,6 +233,28 @@ int32_t csa2_sparse_attn_fp4(const uint16_t* q, const csa2_rows* codes, const cs
                              void* ws, size_t ws_bytes, int32_t* status, void* stream);
 size_t csa2_sparse_attn_workspace(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
 
+/* csa2_sparse_attn_fp4_local: csa2_sparse_attn_fp4 for a layer that keeps its
+ * own cache of the most recent tokens beside the FP4 main cache (V4 kept a
+ * separate per-layer local KV of the latest 128 tokens besides the global KV,
+ * and V4.1 keeps that local cache while a session is active: "How DeepSeek
+ * V4.1 Flash Actually Works", the three KV-cache optimizations, item 3).  The
+ * window positions are read from it, every other position of S from the FP4
+ * cache.  The pages give the local cache no format; here it holds bf16 rows.
+ *   local_kv  bf16 rows of D values (row_bytes >= 2 D, a multiple of 16),
+ *             contiguous (page_table NULL); seq_rows = R >= window is the
+ *             ring length: position p of sequence s is row s*R + (p mod R).
+ *             The caller keeps it current: for every query it holds the
+ *             rows of that query's window positions.
+ * Other arguments, the workspace (csa2_sparse_attn_workspace) and errors as
+ * csa2_sparse_attn_fp4; a local_kv of the wrong shape is CSA2_ERR_INVALID_ARG.
+ */
+int32_t csa2_sparse_attn_fp4_local(const uint16_t* q, const csa2_rows* codes, const csa2_rows* scales,
+                                   const csa2_rows* local_kv, const int32_t* seq_of_query,
+                                   const int32_t* query_pos, const int32_t* sel_idx, const int32_t* sel_cnt,
+                                   int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window,
+                                   float softmax_scale, uint16_t* out, float* lse,
+                                   void* ws, size_t ws_bytes, int32_t* status, void* stream);
+
 /* ------------------------------------------------------------ steps 1-5 as a plan
  * csa2_layer_plan: one decode step through L layers of modes FULL, REINDEX or
  * REUSE ("Full -> Reindex -> Reuse pipeline": "DeepSeek V4.1-Flash: 552B runs
@@ -256,6 +278,9 @@ typedef struct csa2_layer {
   int32_t* pool_cnt;        /* FULL: [nq] out or NULL            */
   int32_t* sel_idx;         /* FULL/REINDEX: [nq][K] out or NULL */
   int32_t* sel_cnt;         /* FULL/REINDEX: [nq] out or NULL    */
+  csa2_rows local_kv;       /* the layer's local window cache (see
+                               csa2_sparse_attn_fp4_local); base NULL: the
+                               window reads the FP4 cache           */
 } csa2_layer;
 
 typedef struct csa2_plan_shape {

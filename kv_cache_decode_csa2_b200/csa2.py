@@ -44,7 +44,8 @@ class csa2_layer(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("w", ctypes.c_void_p), ("keys", csa2_rows),
                 ("q_attn", ctypes.c_void_p), ("codes", csa2_rows), ("scales", csa2_rows),
                 ("out", ctypes.c_void_p), ("lse", ctypes.c_void_p), ("pool_idx", ctypes.c_void_p),
-                ("pool_cnt", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p)]
+                ("pool_cnt", ctypes.c_void_p), ("sel_idx", ctypes.c_void_p), ("sel_cnt", ctypes.c_void_p),
+                ("local_kv", csa2_rows)]
 
 
 class csa2_plan_shape(ctypes.Structure):
@@ -70,6 +71,8 @@ _SIGS = {
     "csa2_sparse_attn_fp4": (_I32, [_P, _RP, _RP, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _F, _P,
                                     _P, _P, _SZ, _P, _P]),
     "csa2_sparse_attn_workspace": (_SZ, [_I32, _I32, _I32, _I32, _I32]),
+    "csa2_sparse_attn_fp4_local": (_I32, [_P, _RP, _RP, _RP, _P, _P, _P, _P, _I32, _I32, _I32, _I32, _I32, _F,
+                                          _P, _P, _P, _SZ, _P, _P]),
     "csa2_layer_plan": (_I32, [_P, _I32, ctypes.POINTER(csa2_layer), ctypes.POINTER(csa2_plan_shape), _P,
                                _SZ, _P, _P]),
     "csa2_layer_plan_workspace": (_SZ, [_P, _I32, ctypes.POINTER(csa2_plan_shape)]),
@@ -233,8 +236,11 @@ def csa2_reindex(q, w, keys: Rows, pool_idx, pool_cnt, K: int, sel_idx, *, sel_c
 
 def csa2_sparse_attn_fp4(q, codes: Rows, scales: Rows, query_pos, sel_idx, out, *, sel_cnt=None,
                          seq_of_query=None, window: int = 128, softmax_scale: float = 0.0, lse=None,
-                         status=None, ws=None, stream=None):
-    """Attention over selection U window on the FP4 cache.  q bf16 [nq][Hq][D]."""
+                         local_kv: Rows | None = None, status=None, ws=None, stream=None):
+    """Attention over selection U window on the FP4 cache.  q bf16 [nq][Hq][D].
+    With ``local_kv`` (bf16 rows [n_seq * R][D], ``seq_rows`` = R >= window)
+    the window rows come from the layer's local cache
+    (csa2_sparse_attn_fp4_local)."""
     L = lib()
     _dev(q, torch.bfloat16, "q")
     _dev(out, torch.bfloat16, "out")
@@ -244,11 +250,15 @@ def csa2_sparse_attn_fp4(q, codes: Rows, scales: Rows, query_pos, sel_idx, out, 
     need = L.csa2_sparse_attn_workspace(nq, Hq, D, K, window)
     ws = _workspace(need, q.device) if ws is None else ws
     cr, sr = codes.c(), scales.c()
-    code = L.csa2_sparse_attn_fp4(_ptr(q), ctypes.byref(cr), ctypes.byref(sr), _ptr(seq_of_query),
-                                  _ptr(query_pos), _ptr(sel_idx), _ptr(sel_cnt), nq, Hq, D, K, window,
-                                  softmax_scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(status),
-                                  _stream(stream))
-    _check(code, "csa2_sparse_attn_fp4")
+    tail = (_ptr(seq_of_query), _ptr(query_pos), _ptr(sel_idx), _ptr(sel_cnt), nq, Hq, D, K, window,
+            softmax_scale, _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _ptr(status), _stream(stream))
+    if local_kv is None:
+        code = L.csa2_sparse_attn_fp4(_ptr(q), ctypes.byref(cr), ctypes.byref(sr), *tail)
+        _check(code, "csa2_sparse_attn_fp4")
+    else:
+        lr = local_kv.c()
+        code = L.csa2_sparse_attn_fp4_local(_ptr(q), ctypes.byref(cr), ctypes.byref(sr), ctypes.byref(lr), *tail)
+        _check(code, "csa2_sparse_attn_fp4_local")
     return status
 
 
@@ -280,6 +290,7 @@ class Layer:
     pool_cnt: torch.Tensor | None = None
     sel_idx: torch.Tensor | None = None
     sel_cnt: torch.Tensor | None = None
+    local_kv: Rows | None = None     # the layer's local window cache (bf16 ring of seq_rows rows)
 
 
 class LayerPlan:
@@ -305,6 +316,8 @@ class LayerPlan:
             c.out, c.lse = _ptr(ly.out), _ptr(ly.lse)
             c.pool_idx, c.pool_cnt = _ptr(ly.pool_idx), _ptr(ly.pool_cnt)
             c.sel_idx, c.sel_cnt = _ptr(ly.sel_idx), _ptr(ly.sel_cnt)
+            if ly.local_kv is not None:
+                c.local_kv = ly.local_kv.c()
         s = csa2_plan_shape()
         s.nq, s.H, s.D_idx, s.Hq, s.D, s.P, s.K = nq, H, D_idx, Hq, D, P, K
         s.window, s.max_ctx, s.softmax_scale = window, max_ctx, softmax_scale

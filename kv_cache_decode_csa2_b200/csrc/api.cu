@@ -103,7 +103,7 @@ const char* csa2_status_string(int32_t s) {
   }
 }
 
-int32_t csa2_version(void) { return 100; }   // 0.1.0
+int32_t csa2_version(void) { return 200; }   // 0.2.0: csa2_layer gained local_kv
 
 size_t csa2_trace_table_bytes(void) {
   return (size_t)kTraceKernels * kTraceCtas * kTracePhases * 2 * sizeof(uint64_t);
@@ -235,20 +235,47 @@ static int32_t check_attn(const uint16_t* q, const csa2_rows* codes, const csa2_
   return CSA2_OK;
 }
 
+// A local window cache: contiguous bf16 rows of D values, a ring of at least
+// `window` rows per sequence.
+static bool local_ok(const csa2_rows* v, int32_t D, int32_t window) {
+  return rows_ok(v, 2 * (int64_t)D, 16) && !v->page_table && v->seq_rows >= window;
+}
+
+static int32_t run_attn(const uint16_t* q, const csa2_rows* codes, const csa2_rows* scales,
+                        const csa2_rows* local_kv, const int32_t* seq_of_query, const int32_t* query_pos,
+                        const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq, int32_t Hq, int32_t D,
+                        int32_t K, int32_t window, float softmax_scale, uint16_t* out, float* lse, void* ws,
+                        size_t ws_bytes, int32_t* status, void* stream) {
+  int32_t r = check_attn(q, codes, scales, query_pos, nq, Hq, D, K, window, out);
+  if (r != CSA2_OK) return r;
+  if (!status || (K > 0 && !sel_idx)) return CSA2_ERR_INVALID_ARG;
+  if (local_kv && !local_ok(local_kv, D, window)) return CSA2_ERR_INVALID_ARG;
+  if (!ws || !aligned(ws, 256) || ws_bytes < csa2_sparse_attn_workspace(nq, Hq, D, K, window))
+    return CSA2_ERR_WORKSPACE;
+  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
+  return cuda_status(launch_sparse_attn(q, *codes, *scales, local_kv, seq_of_query, query_pos, sel_idx, sel_cnt,
+                                        nq, Hq, D, K, window, scale, out, lse, ws, ws_bytes, status,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
 int32_t csa2_sparse_attn_fp4(const uint16_t* q, const csa2_rows* codes, const csa2_rows* scales,
                              const int32_t* seq_of_query, const int32_t* query_pos,
                              const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq, int32_t Hq,
                              int32_t D, int32_t K, int32_t window, float softmax_scale, uint16_t* out,
                              float* lse, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
-  int32_t r = check_attn(q, codes, scales, query_pos, nq, Hq, D, K, window, out);
-  if (r != CSA2_OK) return r;
-  if (!status || (K > 0 && !sel_idx)) return CSA2_ERR_INVALID_ARG;
-  if (!ws || !aligned(ws, 256) || ws_bytes < csa2_sparse_attn_workspace(nq, Hq, D, K, window))
-    return CSA2_ERR_WORKSPACE;
-  const float scale = softmax_scale > 0.f ? softmax_scale : 1.0f / sqrtf((float)D);
-  return cuda_status(launch_sparse_attn(q, *codes, *scales, seq_of_query, query_pos, sel_idx, sel_cnt, nq,
-                                        Hq, D, K, window, scale, out, lse, ws, ws_bytes, status,
-                                        static_cast<cudaStream_t>(stream)));
+  return run_attn(q, codes, scales, nullptr, seq_of_query, query_pos, sel_idx, sel_cnt, nq, Hq, D, K, window,
+                  softmax_scale, out, lse, ws, ws_bytes, status, stream);
+}
+
+int32_t csa2_sparse_attn_fp4_local(const uint16_t* q, const csa2_rows* codes, const csa2_rows* scales,
+                                   const csa2_rows* local_kv, const int32_t* seq_of_query,
+                                   const int32_t* query_pos, const int32_t* sel_idx, const int32_t* sel_cnt,
+                                   int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window,
+                                   float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
+                                   int32_t* status, void* stream) {
+  if (!local_kv) return CSA2_ERR_INVALID_ARG;
+  return run_attn(q, codes, scales, local_kv, seq_of_query, query_pos, sel_idx, sel_cnt, nq, Hq, D, K, window,
+                  softmax_scale, out, lse, ws, ws_bytes, status, stream);
 }
 
 // ------------------------------------------------------------------ layer plan
@@ -318,6 +345,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
     int32_t r = check_attn(ly.q_attn, &ly.codes, &ly.scales, s->query_pos, s->nq, s->Hq, s->D, s->K,
                            s->window, ly.out);
     if (r != CSA2_OK) return r;
+    if (ly.local_kv.base && !local_ok(&ly.local_kv, s->D, s->window)) return CSA2_ERR_INVALID_ARG;
     if (modes[i] != CSA2_REUSE) {
       if (!ly.q || !ly.w || !aligned(ly.q, 16)) return CSA2_ERR_INVALID_ARG;
       if (s->D_idx != 64 && s->D_idx != 128) return CSA2_ERR_UNSUPPORTED;
@@ -421,7 +449,8 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
           return CSA2_ERR_CUDA;
       }
     }
-    jobs[i] = AttnJobDesc{ly.q_attn, &ly.codes, &ly.scales, sel_of[i], sel_cnt_of[i], ly.out, ly.lse};
+    jobs[i] = AttnJobDesc{ly.q_attn, &ly.codes,  &ly.scales, sel_of[i], sel_cnt_of[i],
+                          ly.out,    ly.lse,     ly.local_kv.base ? &ly.local_kv : nullptr};
   }
   const float scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->D);
   return cuda_status(launch_sparse_attn_jobs(jobs, L, s->seq_of_query, s->query_pos, s->nq, s->Hq, s->D, s->K,

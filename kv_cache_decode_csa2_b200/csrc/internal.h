@@ -175,10 +175,10 @@ cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, co
                                   int32_t D, int32_t P, int32_t K, const ReindexSelScratch& r,
                                   int32_t* status, cudaStream_t st);
 
-// K4: FP4 sparse attention.
+// K4: FP4 sparse attention (local_kv: the layer's local window cache, or nullptr).
 size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
 cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,
-                               const int32_t* seq_of_query, const int32_t* query_pos,
+                               const csa2_rows* local_kv, const int32_t* seq_of_query, const int32_t* query_pos,
                                const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq,
                                int32_t Hq, int32_t D, int32_t K, int32_t window, float scale,
                                uint16_t* out, float* lse, void* ws, size_t ws_bytes,
@@ -228,6 +228,7 @@ struct AttnJobDesc {
   const int32_t* sel_cnt;
   uint16_t* out;
   float* lse;
+  const csa2_rows* local_kv = nullptr;   // the layer's local window cache (bf16 ring), or none
 };
 constexpr int kMaxAttnJobs = 16;
 void attn_bar_region(void* ws, int32_t n_jobs, int32_t nq, int32_t Hq, int32_t D, void** ptr, size_t* bytes);

@@ -21,6 +21,14 @@
 // columns [r D / kCl, (r + 1) D / kCl) of every head; otherwise a merge kernel
 // does the same.  Several layers of a plan go into one launch (a job array),
 // so independent layers run side by side.
+//
+// A layer may keep its own cache of the most recent tokens beside the FP4
+// main cache ("How DeepSeek V4.1 Flash Actually Works", the three KV-cache
+// optimizations, item 3: V4 kept a separate per-layer local KV of the latest
+// 128 tokens, and V4.1 keeps it while a session is active).  Its rows are
+// bf16, in a ring of R >= window rows per sequence (position p in slot
+// p mod R).  The LOCAL instantiation reads the window rows from that ring
+// with 16-byte loads and the selection rows from the FP4 cache.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -52,6 +60,14 @@ struct AttnJob {
   float* lse;
 };
 
+// A job's local window cache (LOCAL instantiation; base nullptr: none).
+struct AttnLocal {
+  const uint8_t* base;
+  int64_t row_bytes;
+  int64_t ring;     // rows per sequence: position p of sequence s is row s ring + p mod ring
+  int64_t n_rows;   // rows in the buffer
+};
+
 struct AttnArgs {
   AttnJob jobs[kMaxJobs];
   const int32_t* seq_of_query;
@@ -63,7 +79,9 @@ struct AttnArgs {
   uint32_t* bar;      // [groups]               barrier counts (zeroed before a fused launch)
   int32_t fused;      // the group merges in the same launch
   int32_t* status;
+  AttnLocal local[kMaxJobs];
 };
+static_assert(sizeof(AttnArgs) <= 4096, "kernel parameters");
 
 // Two E2M1 codes (low nibble = first element) -> f16x2, exactly (every E2M1
 // value is an f16 value).
@@ -203,7 +221,7 @@ __device__ __forceinline__ void merge_slice(const AttnArgs& a, const AttnJob& J,
     J.lse[(size_t)q * a.Hq + h0 + tid] = (Mh[tid] + log2f(Lh[tid])) * 0.69314718055994531f;
 }
 
-template <int D, int HG, int NTHR>
+template <int D, int HG, int NTHR, bool LOCAL>
 __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_constant__ AttnArgs a) {
   using L = AttnSmem<D, HG>;
   constexpr int NW = NTHR / 32;                      // warps
@@ -302,7 +320,21 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
           p = wstart + o0 + (r - ns);
         }
       }
-      if (p >= 0) {
+      bool in_ring = false;   // a window row read from the layer's local cache
+      if constexpr (LOCAL) {
+        const AttnLocal& lw = a.local[job_i];
+        if (p >= 0 && lw.base && r >= ns) {
+          in_ring = true;
+          const int64_t lr = (int64_t)seq * lw.ring + p % lw.ring;
+          if (lr < 0 || lr >= lw.n_rows) {
+            record_error(a.status, CSA2_ERR_INDEX_RANGE);
+            p = -1;
+          } else {
+            cr = -2 - lr;   // ring rows are coded below -1; the FP4 pass leaves them to the ring pass
+          }
+        }
+      }
+      if (p >= 0 && !in_ring) {
         cr = map_row(J.cmap, seq, p);
         sr = map_row(J.smap, seq, p);
         if (cr < 0 || sr < 0) {
@@ -338,6 +370,35 @@ __global__ void __launch_bounds__(NTHR, 1) sparse_attn_kernel(const __grid_const
         uint32_t packed[4];
         dequant8(cw[u], sb[u], packed);
         *reinterpret_cast<uint4*>(kv_s + r * L::kKV + g * 16) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+      if constexpr (LOCAL) {
+        // ring rows: the bf16 values as they are, four 16-byte loads in flight
+        // per thread; the same thread wrote zeros at these items just above
+        const AttnLocal& lw = a.local[job_i];
+        if (lw.base) {
+          constexpr int CH = 4;
+#pragma unroll
+          for (int u0 = 0; u0 < DPER; u0 += CH) {
+            int4 v[CH];
+            int64_t at[CH];
+#pragma unroll
+            for (int c = 0; c < CH; ++c) {
+              at[c] = -1;
+              const int u = u0 + c;
+              if (u < DPER) {
+                const int i = tid + u * NTHR, r = i / (D / 8), g = i % (D / 8);
+                const int64_t cr = row_s[r];
+                if (cr <= -2) {
+                  v[c] = __ldg(reinterpret_cast<const int4*>(lw.base + (-2 - cr) * lw.row_bytes) + g);
+                  at[c] = (int64_t)r * L::kKV + g * 16;
+                }
+              }
+            }
+#pragma unroll
+            for (int c = 0; c < CH; ++c)
+              if (at[c] >= 0) *reinterpret_cast<int4*>(kv_s + at[c]) = v[c];
+          }
+        }
       }
     }
     __syncthreads();
@@ -487,19 +548,20 @@ __global__ void __launch_bounds__(NTHR) attn_merge_kernel(const __grid_constant_
   merge_slice<D, HG, NTHR>(a, a.jobs[job_i], q, blockIdx.y * HG, gidx, blockIdx.x, tab);
 }
 
-template <int D, int HG, int NTHR>
+template <int D, int HG, int NTHR, bool LOCAL>
 cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
   using L = AttnSmem<D, HG>;
   static SetupMask done{0};
   static std::atomic<int> max_ctas[64];   // co-resident CTAs per device (0: not yet known)
-  cudaError_t e = ensure_smem(sparse_attn_kernel<D, HG, NTHR>, (int)L::total, done);
+  cudaError_t e = ensure_smem(sparse_attn_kernel<D, HG, NTHR, LOCAL>, (int)L::total, done);
   if (e != cudaSuccess) return e;
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 64 && !max_ctas[dev]) {
     int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_attn_kernel<D, HG, NTHR>, NTHR, L::total);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, sparse_attn_kernel<D, HG, NTHR, LOCAL>, NTHR,
+                                                      L::total);
     if (e != cudaSuccess) return e;
     max_ctas[dev] = per_sm * sm_count();
   }
@@ -511,9 +573,10 @@ cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
       e = cudaMemsetAsync(a.bar, 0, (size_t)grid.y * grid.z * sizeof(uint32_t), st);
       if (e != cudaSuccess) return e;
     }
-    return launch_k(sparse_attn_kernel<D, HG, NTHR>, grid, dim3(NTHR), L::total, st, true, launch_opts().pdl, a);
+    return launch_k(sparse_attn_kernel<D, HG, NTHR, LOCAL>, grid, dim3(NTHR), L::total, st, true,
+                    launch_opts().pdl, a);
   }
-  sparse_attn_kernel<D, HG, NTHR><<<grid, NTHR, L::total, st>>>(a);
+  sparse_attn_kernel<D, HG, NTHR, LOCAL><<<grid, NTHR, L::total, st>>>(a);
   attn_merge_kernel<D, HG, NTHR><<<grid, NTHR, 0, st>>>(a);
   return cudaGetLastError();
 }
@@ -558,6 +621,7 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
   a.n_jobs = n_jobs;
   a.scale_log2 = scale * 1.4426950408889634f;
   a.status = status;
+  bool any_local = false;
   for (int j = 0; j < n_jobs; ++j) {
     AttnJob& J = a.jobs[j];
     J.q = jobs[j].q;
@@ -571,6 +635,11 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
     J.sel_cnt = jobs[j].sel_cnt;
     J.out = jobs[j].out;
     J.lse = jobs[j].lse;
+    const csa2_rows* lk = jobs[j].local_kv;
+    a.local[j] = lk && lk->base ? AttnLocal{static_cast<const uint8_t*>(lk->base), lk->row_bytes, lk->seq_rows,
+                                            lk->n_rows}
+                                : AttnLocal{nullptr, 0, 1, 0};
+    any_local |= a.local[j].base != nullptr;
   }
   const int HG = Hq <= 16 ? 16 : kAttnHG;
   const size_t groups = (size_t)n_jobs * nq * ((Hq + HG - 1) / HG);
@@ -578,17 +647,23 @@ cudaError_t launch_sparse_attn_jobs(const AttnJobDesc* jobs, int n_jobs, const i
   a.part_o = c.take<float>(groups * kCl * HG * D);
   a.part_ml = c.take<float2>(groups * kCl * HG);
   a.bar = c.take<uint32_t>(groups);
-  if (D == 512) return HG == 16 ? launch_attn_t<512, 16, 256>(a, st) : launch_attn_t<512, kAttnHG, 256>(a, st);
-  return HG == 16 ? launch_attn_t<128, 16, 256>(a, st) : launch_attn_t<128, kAttnHG, 256>(a, st);
+  if (any_local) {
+    if (D == 512)
+      return HG == 16 ? launch_attn_t<512, 16, 256, true>(a, st) : launch_attn_t<512, kAttnHG, 256, true>(a, st);
+    return HG == 16 ? launch_attn_t<128, 16, 256, true>(a, st) : launch_attn_t<128, kAttnHG, 256, true>(a, st);
+  }
+  if (D == 512)
+    return HG == 16 ? launch_attn_t<512, 16, 256, false>(a, st) : launch_attn_t<512, kAttnHG, 256, false>(a, st);
+  return HG == 16 ? launch_attn_t<128, 16, 256, false>(a, st) : launch_attn_t<128, kAttnHG, 256, false>(a, st);
 }
 
 cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,
-                               const int32_t* seq_of_query, const int32_t* query_pos,
+                               const csa2_rows* local_kv, const int32_t* seq_of_query, const int32_t* query_pos,
                                const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq,
                                int32_t Hq, int32_t D, int32_t K, int32_t window, float scale,
                                uint16_t* out, float* lse, void* ws, size_t /*ws_bytes*/,
                                int32_t* status, cudaStream_t st) {
-  AttnJobDesc j{q, &codes, &scales, sel_idx, sel_cnt, out, lse};
+  AttnJobDesc j{q, &codes, &scales, sel_idx, sel_cnt, out, lse, local_kv};
   return launch_sparse_attn_jobs(&j, 1, seq_of_query, query_pos, nq, Hq, D, K, window, scale, ws,
                                  status, st);
 }

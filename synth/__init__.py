@@ -178,6 +178,26 @@ def kv_values(wl: Workload, layer: int, seq: int, row0: int = 0, row1: int | Non
     return _chunked(fill, n, row0, row1, wl.attn_dim, np.float32)
 
 
+def local_kv_values(wl: Workload, layer: int, seq: int, row0: int, row1: int) -> np.ndarray:
+    """float32 [row1-row0][attn_dim] rows of a layer's local window cache for
+    positions row0..row1-1 of one sequence: the same distribution as
+    kv_values (its own stream: the local rows are not the main cache's
+    values), rounded to the nearest bf16 value, the format the local cache
+    stores."""
+    n = int(wl.lengths()[seq])
+    period = int(round(1.0 / wl.outlier_p)) if wl.outlier_p > 0 else 0
+
+    def fill(c: int, rows: int) -> np.ndarray:
+        g = _gen(wl, "local_kv", layer, seq, c)
+        x = g.standard_normal((rows, wl.attn_dim), dtype=np.float32)
+        if period:
+            hit = g.integers(0, period, size=(rows, wl.attn_dim), dtype=np.uint16) == 0
+            x[hit] *= np.float32(wl.outlier_mul)
+        return x
+
+    return round_to_bf16(_chunked(fill, n, row0, row1, wl.attn_dim, np.float32))
+
+
 def attn_query(wl: Workload, layer: int, query: int) -> np.ndarray:
     """float32 [attn_heads][attn_dim] N(0,1) query, already rounded to the
     nearest bf16 value (ties to even), so it is exactly a bf16 tensor."""

@@ -30,7 +30,7 @@ def test_library_exports_every_declared_function():
 
 def test_version_and_status_strings():
     L = K.lib()
-    assert L.csa2_version() == 100
+    assert L.csa2_version() == 200
     for code in range(9):
         assert L.csa2_status_string(code)
     assert L.csa2_status_string(6) == b"position, page or row out of range"
@@ -96,6 +96,31 @@ def test_rejects_bad_arguments_before_any_launch():
                                   512, 8, 128, 0.0, 16, None, 256, 1 << 20, 16, None) == 2
     # quantiser: D not a multiple of 32
     assert L.csa2_fp4_quantize(16, 4, 48, 48, None, 16, 32, 16, 2, 4, 16, None) == 2
+
+
+def test_local_window_cache_is_checked():
+    L = K.lib()
+    codes, scales = _rows(row_bytes=256), _rows(row_bytes=16)
+    args = (None, 16, 16, None, 1, 64, 512, 8, 128, 0.0, 16, None, 256, 1 << 20, 16, None)
+
+    def call(local):
+        return L.csa2_sparse_attn_fp4_local(16, ctypes.byref(codes), ctypes.byref(scales),
+                                            ctypes.byref(local) if local is not None else None, *args)
+
+    ring = _rows(row_bytes=1024, n_rows=256)
+    ring.seq_rows = 128
+    assert call(ring) == 3                       # a good ring: only the (too small) workspace is left
+    assert call(None) == 1                       # the local entry point needs the cache
+    ring.seq_rows = 127                          # a ring shorter than the 128-row window
+    assert call(ring) == 1
+    ring.seq_rows, ring.row_bytes = 128, 512     # rows shorter than D bf16 values
+    assert call(ring) == 1
+    ring.row_bytes = 1024
+    ring.page_table, ring.page_rows, ring.max_pages = 16, 64, 4   # a ring is not paged
+    assert call(ring) == 1
+    # the same call through the plain entry point with a bad head count still says so first
+    assert L.csa2_sparse_attn_fp4(16, ctypes.byref(codes), ctypes.byref(scales), None, 16, 16, None, 1, 12,
+                                  512, 8, 128, 0.0, 16, None, 256, 1 << 20, 16, None) == 2
 
 
 def test_plan_rejects_reindex_first():

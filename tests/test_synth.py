@@ -29,6 +29,11 @@ def test_distributions():
     assert 0.004 < big.mean() < 0.009
     qa = synth.attn_query(wl, 0, 0)
     assert np.array_equal(qa, synth.round_to_bf16(qa))
+    loc = synth.local_kv_values(wl, 0, 0, 19000, 20000)
+    assert loc.shape == (1000, 512) and np.array_equal(loc, synth.round_to_bf16(loc))
+    assert np.array_equal(synth.local_kv_values(wl, 0, 0, 19500, 19600), loc[500:600])
+    assert not np.array_equal(loc, synth.round_to_bf16(x[19000:20000]))   # not the main cache's values
+    assert 0.5 < np.abs(loc).mean() < 1.2
 
 
 def test_ragged_lengths_and_pages():

@@ -55,7 +55,11 @@ struct ZeroArgs {
   uint32_t words[kMaxZeroRegions];
   int32_t n;
 };
+// The grid after it (the index-score kernel of a plan step) may launch at
+// once: it touches these regions only after its programmatic wait, which
+// returns when this grid has finished and its writes are visible.
 __global__ void __launch_bounds__(256) zero_kernel(const __grid_constant__ ZeroArgs a) {
+  pdl_trigger();
   CSA2_TRACE_BEGIN(kTrZero, threadIdx.x == 0);   // trace point 1: done
   for (int r = 0; r < a.n; ++r)
     for (uint32_t i = blockIdx.x * 256 + threadIdx.x; i < a.words[r]; i += gridDim.x * 256) a.ptr[r][i] = 0u;

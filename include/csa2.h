@@ -319,6 +319,24 @@ int32_t csa2_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_
 const char* csa2_status_string(int32_t status);  /* static string, never NULL */
 int32_t csa2_version(void);                       /* major*10000 + minor*100 + patch */
 
+/* ------------------------------------------------------------ bounded waits
+ * csa2_selftest_wait: a diagnostic of the give-up path of the library's
+ * waits.  Every wait between the CTAs of a kernel (the grid barrier of the
+ * select, reindex and attention kernels) and of the TMA and tensor-core
+ * pipelines (the mbarrier wait) stops after a time limit (2 s in the
+ * kernels), records CSA2_ERR_TIMEOUT and lets its kernel return, so that a
+ * wait which cannot end never hangs the device.  This call runs one such wait
+ * on something that never happens, with a short limit:
+ *   kind 0  the grid barrier, on *counter (device uint32, zeroed by the
+ *           caller; the call adds 1 to it and waits for 2);
+ *   kind 1  the mbarrier wait (counter unused, may be NULL).
+ *   limit_ns  host: how long the wait tries, at most 10^10 (10 s).
+ * After about limit_ns the kernel records CSA2_ERR_TIMEOUT in *status and
+ * returns; the device stays usable.
+ */
+int32_t csa2_selftest_wait(int32_t kind, uint64_t limit_ns, uint32_t* counter, int32_t* status,
+                           void* stream);
+
 /* ------------------------------------------------------------ phase tracing
  * In the traced build of the library (libcsa2_trace.so, compiled with
  * -DCSA2_TRACE) the kernels carry phase markers: one thread of every CTA

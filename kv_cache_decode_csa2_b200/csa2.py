@@ -79,6 +79,7 @@ _SIGS = {
     "csa2_fp4_quantize": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
     "csa2_status_string": (ctypes.c_char_p, [_I32]),
     "csa2_version": (_I32, []),
+    "csa2_selftest_wait": (_I32, [_I32, ctypes.c_uint64, _P, _P, _P]),
     "csa2_trace_table_bytes": (_SZ, []),
     "csa2_trace_attach": (_I32, [_P]),
 }
@@ -272,6 +273,19 @@ def csa2_fp4_quantize(x, codes, scales, *, dst_rows=None, status=None, stream=No
                                _ptr(scales), scales.stride(0), codes.shape[0], _ptr(status),
                                _stream(stream))
     _check(code, "csa2_fp4_quantize")
+    return status
+
+
+def csa2_selftest_wait(kind: int, limit_ns: int, *, counter=None, status=None, stream=None):
+    """Runs one bounded wait that nothing satisfies (kind 0: the grid
+    barrier, on the zeroed int32 ``counter``; kind 1: the mbarrier wait); it
+    records CSA2_ERR_TIMEOUT in ``status`` after about ``limit_ns``."""
+    L = lib()
+    status = new_status() if status is None else status
+    if kind == 0 and counter is None:
+        counter = torch.zeros(1, dtype=torch.int32, device=status.device)
+    _check(L.csa2_selftest_wait(kind, limit_ns, _ptr(counter), _ptr(status), _stream(stream)),
+           "csa2_selftest_wait")
     return status
 
 

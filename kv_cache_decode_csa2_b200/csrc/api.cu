@@ -105,6 +105,12 @@ const char* csa2_status_string(int32_t s) {
 
 int32_t csa2_version(void) { return 200; }   // 0.2.0: csa2_layer gained local_kv
 
+int32_t csa2_selftest_wait(int32_t kind, uint64_t limit_ns, uint32_t* counter, int32_t* status, void* stream) {
+  if (!status || (kind != 0 && kind != 1) || limit_ns > 10000000000ull) return CSA2_ERR_INVALID_ARG;
+  if (kind == 0 && (!counter || !aligned(counter, 4))) return CSA2_ERR_INVALID_ARG;
+  return cuda_status(launch_wait_selftest(kind, limit_ns, counter, status, static_cast<cudaStream_t>(stream)));
+}
+
 size_t csa2_trace_table_bytes(void) {
   return (size_t)kTraceKernels * kTraceCtas * kTracePhases * 2 * sizeof(uint64_t);
 }

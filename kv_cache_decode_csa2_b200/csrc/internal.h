@@ -192,6 +192,10 @@ cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64
 
 int sm_count();
 
+// Self-test of the bounded waits (selftest.cu).
+cudaError_t launch_wait_selftest(int32_t kind, uint64_t limit_ns, uint32_t* counter, int32_t* status,
+                                 cudaStream_t st);
+
 #ifdef CSA2_TRACE
 // The traced build: each translation unit with phase markers sets its table.
 cudaError_t trace_attach_index(uint64_t* table);

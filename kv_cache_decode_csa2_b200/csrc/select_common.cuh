@@ -47,9 +47,10 @@ __device__ __forceinline__ uint64_t sel_scan(uint64_t v, uint64_t* wtmp, uint64_
 // before the launch) reaches `target`, a multiple of G.  The block barrier
 // orders the CTA's writes before thread 0's release-add; thread 0's acquire
 // load, then the block barrier, order the other CTAs' writes before every
-// later read.  Bounded: after kWaitLimitNs it records CSA2_ERR_TIMEOUT and
-// goes on.
-__device__ __forceinline__ void sel_grid_sync(uint32_t* bar, uint32_t target, int32_t* status) {
+// later read.  Bounded: after limit_ns it records CSA2_ERR_TIMEOUT and goes
+// on.
+__device__ __forceinline__ void sel_grid_sync(uint32_t* bar, uint32_t target, int32_t* status,
+                                              uint64_t limit_ns = kWaitLimitNs) {
   __syncthreads();
   if (threadIdx.x == 0) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar) : "memory");
@@ -58,7 +59,7 @@ __device__ __forceinline__ void sel_grid_sync(uint32_t* bar, uint32_t target, in
     if (v < target) {
       const uint64_t t0 = global_ns();
       do {
-        if (global_ns() - t0 > kWaitLimitNs) {
+        if (global_ns() - t0 > limit_ns) {
           record_error(status, CSA2_ERR_TIMEOUT);
           break;
         }

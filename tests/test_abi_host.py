@@ -123,6 +123,14 @@ def test_local_window_cache_is_checked():
                                   512, 8, 128, 0.0, 16, None, 256, 1 << 20, 16, None) == 2
 
 
+def test_wait_selftest_checks_its_arguments():
+    L = K.lib()
+    assert L.csa2_selftest_wait(2, 1000, 16, 16, None) == 1                    # no such kind
+    assert L.csa2_selftest_wait(0, 1000, None, 16, None) == 1                  # the barrier needs a counter
+    assert L.csa2_selftest_wait(1, 1000, None, None, None) == 1                # and every kind a status word
+    assert L.csa2_selftest_wait(1, 10 ** 10 + 1, None, 16, None) == 1          # limits above 10 s are refused
+
+
 def test_plan_rejects_reindex_first():
     L = K.lib()
     modes = (ctypes.c_int32 * 2)(1, 2)

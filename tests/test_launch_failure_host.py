@@ -52,6 +52,12 @@ def test_attention_and_quantiser_report_the_failed_launch():
     assert L.csa2_fp4_quantize(A, 16, 512, 512, None, A, 256, A, 16, 16, A, None) == 4
 
 
+def test_wait_selftest_reports_the_failed_launch():
+    L = K.lib()
+    assert L.csa2_selftest_wait(0, 1000, A, A, None) == 4
+    assert L.csa2_selftest_wait(1, 1000, None, A, None) == 4
+
+
 def test_plan_reports_the_failed_launch():
     L = K.lib()
     modes = (ctypes.c_int32 * 3)(0, 1, 2)

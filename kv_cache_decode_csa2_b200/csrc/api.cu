@@ -7,7 +7,26 @@
 #include "csa2_device.cuh"
 #include "internal.h"
 
+#ifdef CSA2_TRACE
+#include <nvtx3/nvToolsExt.h>
+#endif
+
 using namespace csa2;
+
+// In the traced build every entry point opens a named NVTX range, so that a
+// profiler can attribute each kernel launch to the C call that made it (a
+// plan call nests the calls it makes).  The normal build has none.
+#ifdef CSA2_TRACE
+namespace {
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+};
+}  // namespace
+#define CSA2_API_RANGE(name) ApiRange api_range_(name)
+#else
+#define CSA2_API_RANGE(name) ((void)0)
+#endif
 
 namespace {
 
@@ -141,6 +160,7 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
                         int32_t P, int32_t* pool_idx, int32_t* pool_cnt, int32_t K,
                         int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                         int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_index_full");
   if (!q || !w || !query_pos || !status || !aligned(q, 16)) return CSA2_ERR_INVALID_ARG;
   if (nq < 1 || max_ctx < 1 || P < 0 || K < 0 || P > 65536 || K > 65536) return CSA2_ERR_INVALID_ARG;
   if (nq > 4096) return CSA2_ERR_UNSUPPORTED;   // the index-score kernel's work list holds 4096 queries
@@ -186,6 +206,7 @@ int32_t csa2_topk_pool(const int32_t* scores, int64_t ld, const int32_t* n_valid
                        const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                        int32_t* out_idx, int32_t* out_cnt, void* ws, size_t ws_bytes,
                        int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_topk_pool");
   if (!out_idx || !status || nq < 1 || n_max < 0 || n_max > (1 << 30) || k < 1 || k > 65536)
     return CSA2_ERR_INVALID_ARG;
   if (n_max > 0 && (!scores || ld < n_max)) return CSA2_ERR_INVALID_ARG;
@@ -213,6 +234,7 @@ int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
                      int32_t nq, int32_t H, int32_t D, int32_t P, int32_t K, int32_t* sel_idx,
                      int32_t* sel_cnt, int32_t* scores, void* ws, size_t ws_bytes, int32_t* status,
                      void* stream) {
+  CSA2_API_RANGE("csa2_reindex");
   if (!q || !w || !pool_idx || !pool_cnt || !sel_idx || !status || !aligned(q, 16))
     return CSA2_ERR_INVALID_ARG;
   if (nq < 1 || P < 1 || P > 65536 || K < 1 || K > P) return CSA2_ERR_INVALID_ARG;
@@ -269,6 +291,7 @@ int32_t csa2_sparse_attn_fp4(const uint16_t* q, const csa2_rows* codes, const cs
                              const int32_t* sel_idx, const int32_t* sel_cnt, int32_t nq, int32_t Hq,
                              int32_t D, int32_t K, int32_t window, float softmax_scale, uint16_t* out,
                              float* lse, void* ws, size_t ws_bytes, int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_sparse_attn_fp4");
   return run_attn(q, codes, scales, nullptr, seq_of_query, query_pos, sel_idx, sel_cnt, nq, Hq, D, K, window,
                   softmax_scale, out, lse, ws, ws_bytes, status, stream);
 }
@@ -279,6 +302,7 @@ int32_t csa2_sparse_attn_fp4_local(const uint16_t* q, const csa2_rows* codes, co
                                    int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window,
                                    float softmax_scale, uint16_t* out, float* lse, void* ws, size_t ws_bytes,
                                    int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_sparse_attn_fp4_local");
   if (!local_kv) return CSA2_ERR_INVALID_ARG;
   return run_attn(q, codes, scales, local_kv, seq_of_query, query_pos, sel_idx, sel_cnt, nq, Hq, D, K, window,
                   softmax_scale, out, lse, ws, ws_bytes, status, stream);
@@ -344,6 +368,7 @@ size_t csa2_layer_plan_workspace(const int32_t* modes, int32_t L, const csa2_pla
 int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layers,
                         const csa2_plan_shape* s, void* ws, size_t ws_bytes, int32_t* status,
                         void* stream) {
+  CSA2_API_RANGE("csa2_layer_plan");
   if (!plan_modes_ok(modes, L) || !layers || !s || !status) return CSA2_ERR_INVALID_ARG;
   if (s->P < 1 || s->K < 1 || s->K > s->P || !s->query_pos) return CSA2_ERR_INVALID_ARG;
   for (int i = 0; i < L; ++i) {
@@ -467,6 +492,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
 int32_t csa2_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_x, const int32_t* dst_rows,
                           uint8_t* codes, int64_t ld_codes, uint8_t* scales, int64_t ld_scales,
                           int64_t n_dst_rows, int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_fp4_quantize");
   if (!status || n_rows < 0 || (n_rows > 0 && (!x || !codes || !scales))) return CSA2_ERR_INVALID_ARG;
   if (D < 32 || D > 4096 || D % 32) return CSA2_ERR_UNSUPPORTED;
   if (ld_x < D || ld_x % 4 || !aligned(x, 16) || !aligned(codes, 16) || ld_codes < D / 2 || ld_codes % 16 ||

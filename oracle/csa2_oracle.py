@@ -18,7 +18,8 @@ Sources (web pages on DeepSeek V4.1-Flash; cited by title and section):
        (artofsm.art digest), third paragraph (full / reindex / reuse modes).
   [YS] "How DeepSeek V4.1 Flash Actually Works: A Deep Dive"
        (youtubesummary.com), section "The three KV-cache optimizations",
-       item 2 "Compress Sparse Attention / CA2".
+       item 2 "Compress Sparse Attention / CA2" and item 3 (deployment-time
+       cache management: the per-layer local cache of the latest tokens).
   [DA] "DeepSeek Has Done It Again..." (youtubesummary.com), section
        "Architecture and inference efficiency", bullet "Sparse attention for
        long context".

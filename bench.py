@@ -69,6 +69,38 @@ def peaks() -> dict:
         return {"hbm_gbs": 6650.0, "src": "fallback"}
 
 
+def device_facts(dev) -> dict:
+    """The device's L2 size, and a read-only HBM stream rate measured here:
+    torch.sum over 2 GiB of fp32 (larger than L2), best of 5 after one warm-up,
+    CUDA events.  It is a reference beside the copy peak, not the roofline's
+    denominator.  Runs after the timed region; anything that fails is None."""
+    out = {"l2_bytes": None, "read_only_gbs": None, "read_only_how": "torch.sum of 2 GiB fp32, best of 5"}
+    if getattr(dev, "type", None) != "cuda":
+        return out
+    try:
+        out["l2_bytes"] = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0)) or None
+    except Exception:
+        pass
+    try:
+        x = torch.ones(1 << 29, dtype=torch.float32, device=dev)
+        best = None
+        for i in range(6):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            x.sum()
+            b.record()
+            b.synchronize()
+            if i:
+                ms = a.elapsed_time(b)
+                best = ms if best is None else min(best, ms)
+        del x
+        if best:
+            out["read_only_gbs"] = (1 << 31) / (best / 1e3) / 1e9
+    except Exception:
+        pass
+    return out
+
+
 # ----------------------------------------------------------------- distributed plumbing
 def dist_init(n_gpus: int):
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -507,6 +539,7 @@ def run_gpu(args, rank, world, local):
                     "d2h_bytes_per_step": d2h_bytes, "path": "pinned H2D + csa2_layer_plan + D2H, no graph"},
             "gpu_launches": kernels_per_step(wl) * args.steps,
             "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
+    line["device"] = device_facts(dev)
     if rank == 0 and not args.no_cpu_baseline:
         sec, _ = OracleStep(wl, host).run(1, 0)
         line["cpu_baseline"] = {"value": 1.0 / sec, "unit": "steps/s", "cores": cpu_cores_used(), "kind": "oracle",

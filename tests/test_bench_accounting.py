@@ -63,3 +63,10 @@ def test_window_overlap_is_counted_once():
 
 def test_five_launches_per_decode_step():
     assert _bench().kernels_per_step(synth.C2_1M_PLAN) == 5
+
+
+def test_device_facts_without_a_gpu_are_none():
+    import torch
+    bench = _bench()
+    f = bench.device_facts(torch.device("cpu"))
+    assert f["l2_bytes"] is None and f["read_only_gbs"] is None and "2 GiB" in f["read_only_how"]

@@ -314,6 +314,14 @@ int32_t csa2_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_
                           const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes,
                           uint8_t* scales, int64_t ld_scales, int64_t n_dst_rows,
                           int32_t* status, void* stream);
+/* csa2_fp4_quantize_bf16: the same for bf16 rows (x: bf16 bit patterns as
+ * uint16, ld_x a multiple of 8), the format a layer produces its KV in.  A
+ * bf16 value is exactly a float, so both calls store the same codes for the
+ * same values. */
+int32_t csa2_fp4_quantize_bf16(const uint16_t* x, int64_t n_rows, int32_t D, int64_t ld_x,
+                               const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes,
+                               uint8_t* scales, int64_t ld_scales, int64_t n_dst_rows,
+                               int32_t* status, void* stream);
 
 /* ------------------------------------------------------------ helpers */
 const char* csa2_status_string(int32_t status);  /* static string, never NULL */

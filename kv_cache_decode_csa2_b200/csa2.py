@@ -77,6 +77,7 @@ _SIGS = {
                                _SZ, _P, _P]),
     "csa2_layer_plan_workspace": (_SZ, [_P, _I32, ctypes.POINTER(csa2_plan_shape)]),
     "csa2_fp4_quantize": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
+    "csa2_fp4_quantize_bf16": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
     "csa2_status_string": (ctypes.c_char_p, [_I32]),
     "csa2_version": (_I32, []),
     "csa2_selftest_wait": (_I32, [_I32, ctypes.c_uint64, _P, _P, _P]),
@@ -264,15 +265,17 @@ def csa2_sparse_attn_fp4(q, codes: Rows, scales: Rows, query_pos, sel_idx, out, 
 
 
 def csa2_fp4_quantize(x, codes, scales, *, dst_rows=None, status=None, stream=None):
-    """Store float32 rows x [n][D] as FP4 codes [*][D/2] and E4M3 scales [*][D/32]."""
+    """Store float32 or bfloat16 rows x [n][D] as FP4 codes [*][D/2] and E4M3 scales [*][D/32]."""
     L = lib()
-    _dev(x, torch.float32, "x")
+    if not x.is_cuda or x.dtype not in (torch.float32, torch.bfloat16) or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a 2-D float32 or bfloat16 CUDA tensor with unit inner stride")
     n, D = x.shape
     status = new_status(x.device) if status is None else status
-    code = L.csa2_fp4_quantize(_ptr(x), n, D, x.stride(0), _ptr(dst_rows), _ptr(codes), codes.stride(0),
-                               _ptr(scales), scales.stride(0), codes.shape[0], _ptr(status),
-                               _stream(stream))
-    _check(code, "csa2_fp4_quantize")
+    fn, name = ((L.csa2_fp4_quantize_bf16, "csa2_fp4_quantize_bf16") if x.dtype == torch.bfloat16
+                else (L.csa2_fp4_quantize, "csa2_fp4_quantize"))
+    code = fn(_ptr(x), n, D, x.stride(0), _ptr(dst_rows), _ptr(codes), codes.stride(0), _ptr(scales),
+              scales.stride(0), codes.shape[0], _ptr(status), _stream(stream))
+    _check(code, name)
     return status
 
 

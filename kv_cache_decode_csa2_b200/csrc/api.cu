@@ -489,17 +489,34 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
 }
 
 // ------------------------------------------------------------------ FP4 cache write
+// Rows of `elem` bytes per value, 16-byte aligned: ld_x a multiple of 16 / elem.
+static int32_t run_fp4_quantize(const void* x, bool bf16, int64_t n_rows, int32_t D, int64_t ld_x,
+                                const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes, uint8_t* scales,
+                                int64_t ld_scales, int64_t n_dst_rows, int32_t* status, void* stream) {
+  const int64_t per16 = bf16 ? 8 : 4;   // values per 16 bytes
+  if (!status || n_rows < 0 || (n_rows > 0 && (!x || !codes || !scales))) return CSA2_ERR_INVALID_ARG;
+  if (D < 32 || D > 4096 || D % 32) return CSA2_ERR_UNSUPPORTED;
+  if (ld_x < D || ld_x % per16 || !aligned(x, 16) || !aligned(codes, 16) || ld_codes < D / 2 || ld_codes % 16 ||
+      ld_scales < D / 32 || n_dst_rows < 1)
+    return CSA2_ERR_INVALID_ARG;
+  return cuda_status(launch_fp4_quantize(x, bf16, n_rows, D, ld_x, dst_rows, codes, ld_codes, scales, ld_scales,
+                                         n_dst_rows, status, static_cast<cudaStream_t>(stream)));
+}
+
 int32_t csa2_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_x, const int32_t* dst_rows,
                           uint8_t* codes, int64_t ld_codes, uint8_t* scales, int64_t ld_scales,
                           int64_t n_dst_rows, int32_t* status, void* stream) {
   CSA2_API_RANGE("csa2_fp4_quantize");
-  if (!status || n_rows < 0 || (n_rows > 0 && (!x || !codes || !scales))) return CSA2_ERR_INVALID_ARG;
-  if (D < 32 || D > 4096 || D % 32) return CSA2_ERR_UNSUPPORTED;
-  if (ld_x < D || ld_x % 4 || !aligned(x, 16) || !aligned(codes, 16) || ld_codes < D / 2 || ld_codes % 16 ||
-      ld_scales < D / 32 || n_dst_rows < 1)
-    return CSA2_ERR_INVALID_ARG;
-  return cuda_status(launch_fp4_quantize(x, n_rows, D, ld_x, dst_rows, codes, ld_codes, scales, ld_scales,
-                                         n_dst_rows, status, static_cast<cudaStream_t>(stream)));
+  return run_fp4_quantize(x, false, n_rows, D, ld_x, dst_rows, codes, ld_codes, scales, ld_scales, n_dst_rows,
+                          status, stream);
+}
+
+int32_t csa2_fp4_quantize_bf16(const uint16_t* x, int64_t n_rows, int32_t D, int64_t ld_x,
+                               const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes, uint8_t* scales,
+                               int64_t ld_scales, int64_t n_dst_rows, int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_fp4_quantize_bf16");
+  return run_fp4_quantize(x, true, n_rows, D, ld_x, dst_rows, codes, ld_codes, scales, ld_scales, n_dst_rows,
+                          status, stream);
 }
 
 }  // extern "C"

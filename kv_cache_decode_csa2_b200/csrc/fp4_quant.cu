@@ -11,6 +11,9 @@
 // scale (4 bits), and amax with 3 * (v_c + v_{c+1}) for adjacent E4M3 values
 // (at most 8 bits).  Every such product is exact in fp32, so no division
 // rounds.  The result is the nearest code of the exact quotient.
+//
+// The input is fp32 or bf16 rows (bf16 widens to fp32 exactly, so both give
+// the codes of the same values).
 #include "csa2_device.cuh"
 #include "internal.h"
 
@@ -55,7 +58,7 @@ __device__ __forceinline__ uint32_t e2m1_code(float x, float s) {
 }
 
 struct QuantArgs {
-  const float* x;
+  const void* x;      // float or bf16 (uint16 bit patterns) rows
   int64_t n_rows, ld_x;
   int32_t D;
   const int32_t* dst_rows;
@@ -67,6 +70,7 @@ struct QuantArgs {
   int32_t* status;
 };
 
+template <bool BF16>
 __global__ void __launch_bounds__(256) fp4_quantize_kernel(const QuantArgs a) {
   const int blocks_per_row = a.D / 32;
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -78,15 +82,29 @@ __global__ void __launch_bounds__(256) fp4_quantize_kernel(const QuantArgs a) {
     record_error(a.status, CSA2_ERR_INDEX_RANGE);
     return;
   }
-  const float4* src = reinterpret_cast<const float4*>(a.x + r * a.ld_x + b * 32);
   float v[32];
+  if constexpr (BF16) {
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + r * a.ld_x + b * 32);
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const float4 f = __ldg(src + k);
-    v[4 * k] = f.x;
-    v[4 * k + 1] = f.y;
-    v[4 * k + 2] = f.z;
-    v[4 * k + 3] = f.w;
+    for (int k = 0; k < 4; ++k) {   // 8 bf16 per load; bf16 bits << 16 is the same value in fp32
+      const uint4 u = __ldg(src + k);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        v[8 * k + 2 * j] = __uint_as_float(w4[j] << 16);
+        v[8 * k + 2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+      }
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + r * a.ld_x + b * 32);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 f = __ldg(src + k);
+      v[4 * k] = f.x;
+      v[4 * k + 1] = f.y;
+      v[4 * k + 2] = f.z;
+      v[4 * k + 3] = f.w;
+    }
   }
   float amax = 0.f;
 #pragma unroll
@@ -104,7 +122,7 @@ __global__ void __launch_bounds__(256) fp4_quantize_kernel(const QuantArgs a) {
 
 }  // namespace
 
-cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_x,
+cudaError_t launch_fp4_quantize(const void* x, bool bf16, int64_t n_rows, int32_t D, int64_t ld_x,
                                 const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes,
                                 uint8_t* scales, int64_t ld_scales, int64_t n_dst_rows,
                                 int32_t* status, cudaStream_t st) {
@@ -112,7 +130,8 @@ cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64
   const int64_t items = n_rows * (D / 32);
   if (items == 0) return cudaSuccess;
   const int64_t grid = (items + 255) / 256;
-  fp4_quantize_kernel<<<(unsigned)grid, 256, 0, st>>>(a);
+  if (bf16) fp4_quantize_kernel<true><<<(unsigned)grid, 256, 0, st>>>(a);
+  else fp4_quantize_kernel<false><<<(unsigned)grid, 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 

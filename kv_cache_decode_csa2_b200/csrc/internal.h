@@ -185,7 +185,7 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const 
                                int32_t* status, cudaStream_t st);
 
 // K7: FP4 quantiser.
-cudaError_t launch_fp4_quantize(const float* x, int64_t n_rows, int32_t D, int64_t ld_x,
+cudaError_t launch_fp4_quantize(const void* x, bool bf16, int64_t n_rows, int32_t D, int64_t ld_x,
                                 const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes,
                                 uint8_t* scales, int64_t ld_scales, int64_t n_dst_rows,
                                 int32_t* status, cudaStream_t st);

@@ -96,6 +96,8 @@ def test_rejects_bad_arguments_before_any_launch():
                                   512, 8, 128, 0.0, 16, None, 256, 1 << 20, 16, None) == 2
     # quantiser: D not a multiple of 32
     assert L.csa2_fp4_quantize(16, 4, 48, 48, None, 16, 32, 16, 2, 4, 16, None) == 2
+    # bf16 rows must start on 16 bytes: ld_x a multiple of 8 values (fp32: of 4)
+    assert L.csa2_fp4_quantize_bf16(16, 4, 64, 68, None, 16, 32, 16, 2, 4, 16, None) == 1
 
 
 def test_local_window_cache_is_checked():

@@ -50,6 +50,7 @@ def test_attention_and_quantiser_report_the_failed_launch():
     assert L.csa2_sparse_attn_fp4_local(A, ctypes.byref(codes), ctypes.byref(scales), ctypes.byref(ring), None, A,
                                         A, A, 1, 64, 512, 512, 128, 0.0, A, None, A, BIG, A, None) == 4
     assert L.csa2_fp4_quantize(A, 16, 512, 512, None, A, 256, A, 16, 16, A, None) == 4
+    assert L.csa2_fp4_quantize_bf16(A, 16, 512, 512, None, A, 256, A, 16, 16, A, None) == 4
 
 
 def test_wait_selftest_reports_the_failed_launch():

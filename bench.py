@@ -26,6 +26,12 @@ prefix with the int8 indexer, keeping its top-512 and attending to them plus
 the 128-row window (one csa2_index_full and one csa2_sparse_attn_fp4 call,
 captured in a CUDA graph per replica).  It prints queries/s and the int8
 TOP/s of the index stage.
+
+    python bench.py --workload quantize [--steps K] [--warmup W]
+
+times the FP4 cache write: 1,048,576 bf16 rows of d512 (one layer's latent KV
+at the 1M context) stored as E2M1 codes and E4M3 scales by
+csa2_fp4_quantize, in rows/s and HBM GB/s.
 """
 from __future__ import annotations
 
@@ -51,6 +57,8 @@ METRIC = "decode steps/s and HBM GB/s (% of B200 roofline) at 1M-token context"
 WL = synth.C2_1M_PLAN
 METRIC_PREFILL = "prefill-chunk queries/s and index int8 TOP/s (2048 causal queries, 262144 context)"
 WL_PREFILL = synth.C4_PREFILL
+METRIC_QUANT = "FP4 cache write rows/s and HBM GB/s (1,048,576 bf16 rows of d512 -> E2M1 + E4M3)"
+QUANT_SAMPLE_ROWS = 16384
 # DRAM bytes (read + write) of one index-score launch on the decode workload,
 # from one ncu capture of this kernel on it (its summary is kept with the
 # profiles); to be reset to None whenever that kernel changes.
@@ -758,6 +766,132 @@ def run_prefill(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- FP4 cache write
+def quant_bytes_per_row(D: int) -> int:
+    """Algorithmic bytes of storing one bf16 row of D values as FP4: the row
+    read (2 D) and the codes (D / 2) and scales (D / 32) written."""
+    return 2 * D + D // 2 + D // 32
+
+
+def oracle_quant_rows_per_s(wl, rows: int) -> tuple[float, str]:
+    """The oracle's FP4 quantiser on the first ``rows`` rows of layer 0 (bf16
+    values), timed on one host core."""
+    import oracle as O
+    from threadpoolctl import threadpool_limits
+    x = synth.round_to_bf16(synth.kv_values(wl, 0, 0, 0, rows))
+    with threadpool_limits(1):
+        t0 = time.perf_counter()
+        O.fp4_quantize(x)
+        t = time.perf_counter() - t0
+    return rows / t, f"{rows} bf16 rows of d{wl.attn_dim} of the same cache, one call"
+
+
+def run_reference_quantize(args, rank, world):
+    if rank != 0:
+        return
+    wl = WL
+    vs = [oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS)[0] for _ in range(max(1, min(args.steps, 3)))]
+    v = sum(vs) / len(vs)
+    line = {"impl": "reference", "metric": METRIC_QUANT, "value": v, "unit": "rows/s", "n_gpus": args.gpus,
+            "steps": len(vs), "warmup": 0, "ms_per_step": 1e3 * (1 << 20) / v, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "fp4_cache_write_1m_rows_d512"},
+            "cpu_baseline": {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{QUANT_SAMPLE_ROWS} rows per step"},
+            "e2e": {"value": v, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_quantize(args, rank, world, local):
+    """A step stores one layer's latent KV at the 1M context, 1,048,576 bf16
+    rows of d512 (1 GiB, far beyond L2), as FP4 codes and E4M3 scales with
+    csa2_fp4_quantize (one launch), replayed in a CUDA graph."""
+    from kv_cache_decode_csa2_b200 import csa2 as B
+    dev = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(dev)
+    wl = WL
+    t_setup = time.time()
+    n, D = int(wl.lengths()[0]), wl.attn_dim
+    status = B.new_status(dev)
+    x = torch.empty((n, D), dtype=torch.bfloat16, device=dev)
+    step_rows = 1 << 17
+    for a in range(0, n, step_rows):
+        b = min(n, a + step_rows)
+        x[a:b] = torch.from_numpy(synth.kv_values(wl, 0, 0, a, b)).to(dev).to(torch.bfloat16)
+    codes = torch.empty((n, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((n, D // 32), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        B.csa2_fp4_quantize(x, codes, scales, status=status, stream=stream)
+    torch.cuda.synchronize()
+    B.check_status(status)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        B.csa2_fp4_quantize(x, codes, scales, status=status, stream=stream)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t_setup
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            g.replay()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id(dev)) as clk:
+        time.sleep(0.3)
+        with torch.cuda.stream(stream):
+            ev0.record(stream)
+            for _ in range(args.steps):
+                g.replay()
+            ev1.record(stream)
+        torch.cuda.synchronize()
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
+    barrier(world)
+    B.check_status(status)
+    per_row = quant_bytes_per_row(D)
+    achieved = n * per_row / (ms / 1e3) / 1e9
+    pk = peaks()
+
+    # end to end: the rows in from pinned host memory, the codes and scales back
+    e_steps = 3
+    xh = x.cpu().pin_memory()
+    ch = torch.empty(codes.shape, dtype=codes.dtype, pin_memory=True)
+    sh = torch.empty(scales.shape, dtype=scales.dtype, pin_memory=True)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(e_steps):
+            x.copy_(xh, non_blocking=True)
+            B.csa2_fp4_quantize(x, codes, scales, status=status, stream=stream)
+            ch.copy_(codes, non_blocking=True)
+            sh.copy_(scales, non_blocking=True)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e_steps
+    B.check_status(status)
+
+    line = {"metric": METRIC_QUANT, "value": world * n / (ms / 1e3), "unit": "rows/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16->fp4", "data": "synthetic",
+            "config": {"workload": "fp4_cache_write_1m_rows_d512", "rows": n, "d": D, "input": "bf16",
+                       "l2": "1 GiB of input per step, far beyond L2", "parallelism": "one cache per rank"},
+            "roofline": {"kernel": "fp4_quantize_kernel<bf16>", "bound": "hbm", "achieved": achieved,
+                         "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
+                         "peak_src": pk["src"], "ms_per_launch": ms, "bytes_per_launch": n * per_row,
+                         "traffic": None},
+            "e2e": {"value": world * n / (e_ms / 1e3), "unit": "rows/s",
+                    "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+                    "d2h_bytes_per_step": ch.numel() + sh.numel(),
+                    "path": "pinned H2D + csa2_fp4_quantize + D2H, no graph"},
+            "gpu_launches": args.steps, "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
+    if rank == 0 and not args.no_cpu_baseline:
+        v, sample = oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS)
+        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle", "sample": sample}
+    del g
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -765,8 +899,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
-                    help="decode: the 1M-context 8-layer step (default); prefill: the 2048-query chunk")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "quantize"],
+                    help="decode: the 1M-context 8-layer step (default); prefill: the 2048-query chunk; "
+                         "quantize: the FP4 cache write of 1M bf16 rows")
     ap.add_argument("--replicas", type=int, default=N_REPLICAS,
                     help="device copies of the state rotated between steps (4 keep each step's reads out of L2)")
     args = ap.parse_args()
@@ -774,7 +909,10 @@ def main():
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_init(args.gpus)
     try:
-        if args.workload == "prefill":
+        if args.workload == "quantize":
+            (run_reference_quantize if args.impl == "reference" else run_quantize)(args, rank, world, *(
+                () if args.impl == "reference" else (local,)))
+        elif args.workload == "prefill":
             (run_reference_prefill if args.impl == "reference" else run_prefill)(args, rank, world, *(
                 () if args.impl == "reference" else (local,)))
         elif args.impl == "reference":

@@ -70,3 +70,9 @@ def test_device_facts_without_a_gpu_are_none():
     bench = _bench()
     f = bench.device_facts(torch.device("cpu"))
     assert f["l2_bytes"] is None and f["read_only_gbs"] is None and "2 GiB" in f["read_only_how"]
+
+
+def test_fp4_cache_write_bytes_per_row():
+    bench = _bench()
+    assert bench.quant_bytes_per_row(512) == 1024 + 256 + 16     # bf16 row in, codes and scales out
+    assert bench.quant_bytes_per_row(128) == 256 + 64 + 4

@@ -288,6 +288,10 @@ typedef struct csa2_plan_shape {
   float softmax_scale;             /* <= 0: 1/sqrt(D) */
   const int32_t* seq_of_query;     /* device [nq] or NULL */
   const int32_t* query_pos;        /* device [nq] */
+  int32_t group_queries;           /* nonzero: consecutive queries of one sequence
+                                      (a speculative-verify block) share each key tile
+                                      of the index scans in groups of four, from 2
+                                      queries on; zero: only from 16 queries on */
 } csa2_plan_shape;
 
 int32_t csa2_layer_plan(const int32_t* modes /* host [L] */, int32_t L,

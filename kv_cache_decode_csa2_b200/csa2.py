@@ -53,7 +53,7 @@ class csa2_plan_shape(ctypes.Structure):
                 ("Hq", ctypes.c_int32), ("D", ctypes.c_int32), ("P", ctypes.c_int32),
                 ("K", ctypes.c_int32), ("window", ctypes.c_int32), ("max_ctx", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("seq_of_query", ctypes.c_void_p),
-                ("query_pos", ctypes.c_void_p)]
+                ("query_pos", ctypes.c_void_p), ("group_queries", ctypes.c_int32)]
 
 
 _P, _I32, _I64, _SZ, _F = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
@@ -315,7 +315,8 @@ class LayerPlan:
     run() is one C call (and can be captured in a CUDA graph)."""
 
     def __init__(self, modes, layers: list[Layer], *, query_pos, max_ctx: int, P: int, K: int,
-                 window: int = 128, seq_of_query=None, softmax_scale: float = 0.0, ws=None):
+                 window: int = 128, seq_of_query=None, softmax_scale: float = 0.0, group_queries: bool = False,
+                 ws=None):
         self.lib = lib()
         self.keep = (layers, query_pos, seq_of_query)
         L = len(modes)
@@ -339,6 +340,7 @@ class LayerPlan:
         s.nq, s.H, s.D_idx, s.Hq, s.D, s.P, s.K = nq, H, D_idx, Hq, D, P, K
         s.window, s.max_ctx, s.softmax_scale = window, max_ctx, softmax_scale
         s.seq_of_query, s.query_pos = _ptr(seq_of_query), _ptr(query_pos)
+        s.group_queries = 1 if group_queries else 0
         self.shape = s
         need = self.lib.csa2_layer_plan_workspace(self.modes, L, ctypes.byref(s))
         if need == 0:

@@ -422,6 +422,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
     n_reindex += modes[i] == CSA2_REINDEX;
   }
   LaunchOpts opts;
+  opts.group = s->group_queries != 0;
   if (n_full == 1 && n_reindex <= kMaxReindexJobs) {
     void* zp[3];
     size_t zb[3];

@@ -553,8 +553,10 @@ cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows
 
   const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
   // Many queries (a prefill chunk) share key tiles in groups of four, with the
-  // histogram left to the top-k; decode keeps one query per segment.
-  const bool grouped = nq >= kGroupMinQueries && N <= 64;
+  // histogram left to the top-k; decode keeps one query per segment.  A plan
+  // call that says its queries come in same-sequence blocks (a verify block)
+  // groups them from two queries on.
+  const bool grouped = N <= 64 && (nq >= kGroupMinQueries || (launch_opts().group && nq >= 2));
   if (hist_built) *hist_built = !grouped && hist;
   IndexArgs a{q, w, seq_of_query, query_pos, to_rowmap(keys), nq, H, max_ctx, scores, ld,
               grouped ? nullptr : hist, status};

@@ -29,10 +29,13 @@ struct Carver {
 //   pdl        launch the index-score, select, reindex and attention kernels
 //              as programmatic dependents of the kernel before them;
 //   prezeroed  the top-k, reindex and attention scratch was zeroed by the
-//              caller (in the kernel launched just before).
+//              caller (in the kernel launched just before);
+//   group      index scans group the queries of a sequence from 2 queries on
+//              (a verify block), not only from 16.
 struct LaunchOpts {
   bool pdl = false;
   bool prezeroed = false;
+  bool group = false;
 };
 LaunchOpts& launch_opts();
 struct LaunchOptsScope {   // sets the options for its lifetime

@@ -152,7 +152,7 @@ size_t csa2_index_full_workspace(int32_t nq, int32_t max_ctx, int32_t P, int32_t
  *             ascending within the valid prefix (CSA2_ERR_ORDER otherwise);
  *             NULL: candidate j is position j
  *   k         wanted count; out_idx int32 [nq][k], out_cnt int32 [nq]
- * Supported: 0 <= n_max <= 2^30, 1 <= k <= 65536.
+ * Supported: 1 <= nq <= 65535, 0 <= n_max <= 2^30, 1 <= k <= 65536.
  */
 int32_t csa2_topk_pool(const int32_t* scores, int64_t ld, const int32_t* n_valid,
                        const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
@@ -196,7 +196,7 @@ int32_t csa2_topk_pool_noalloc(const int32_t* scores, int64_t ld, const int32_t*
  *   pool_idx  int32 [nq][P] ascending positions, pool_cnt int32 [nq]
  *   sel_idx   int32 [nq][K] out, sel_cnt int32 [nq] out
  *   scores    int32 [nq][P] or NULL: score of each pool entry (slot order)
- * Supported: D in {64, 128}; 1 <= H <= 128; 1 <= P <= 65536; 1 <= K <= P.
+ * Supported: D in {64, 128}; 1 <= H <= 128; 1 <= nq <= 65535; 1 <= P <= 65536; 1 <= K <= P.
  */
 int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
                      const int32_t* seq_of_query, const int32_t* pool_idx,
@@ -264,6 +264,8 @@ int32_t csa2_sparse_attn_fp4_local(const uint16_t* q, const csa2_rows* codes, co
  * modes[0] must be FULL.  A REINDEX layer re-scores the pool of the most
  * recent FULL layer.  A REUSE layer attends with the selection of the most
  * recent FULL or REINDEX layer (no index work at all).
+ * Supported: 1 <= L <= 16 layers, nq * L <= 65535 (one attention launch
+ * covers every layer), the per-op limits of the calls above.
  */
 typedef struct csa2_layer {
   const int8_t* q;          /* FULL/REINDEX: int8 [nq][H][D_idx] */

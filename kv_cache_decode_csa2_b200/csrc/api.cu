@@ -210,6 +210,7 @@ int32_t csa2_topk_pool(const int32_t* scores, int64_t ld, const int32_t* n_valid
   if (!out_idx || !status || nq < 1 || n_max < 0 || n_max > (1 << 30) || k < 1 || k > 65536)
     return CSA2_ERR_INVALID_ARG;
   if (n_max > 0 && (!scores || ld < n_max)) return CSA2_ERR_INVALID_ARG;
+  if (nq > 65535) return CSA2_ERR_UNSUPPORTED;   // queries index a grid dimension
   if (ws_bytes < csa2_topk_pool_workspace(nq, n_max, k) || (n_max > kSmallMax && (!ws || !aligned(ws, 256))))
     return CSA2_ERR_WORKSPACE;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -239,7 +240,7 @@ int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
     return CSA2_ERR_INVALID_ARG;
   if (nq < 1 || P < 1 || P > 65536 || K < 1 || K > P) return CSA2_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return CSA2_ERR_UNSUPPORTED;
-  if (H < 1 || H > 128) return CSA2_ERR_UNSUPPORTED;
+  if (H < 1 || H > 128 || nq > 65535) return CSA2_ERR_UNSUPPORTED;
   if (!rows_ok(keys, D, 16)) return CSA2_ERR_INVALID_ARG;
   if (!ws || !aligned(ws, 256) || ws_bytes < csa2_reindex_workspace(nq, P, K)) return CSA2_ERR_WORKSPACE;
   const ReindexJobDesc job{q, w, keys, scores, sel_idx, sel_cnt};
@@ -371,6 +372,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
   CSA2_API_RANGE("csa2_layer_plan");
   if (!plan_modes_ok(modes, L) || !layers || !s || !status) return CSA2_ERR_INVALID_ARG;
   if (s->P < 1 || s->K < 1 || s->K > s->P || !s->query_pos) return CSA2_ERR_INVALID_ARG;
+  if ((int64_t)s->nq * L > 65535) return CSA2_ERR_UNSUPPORTED;   // one attention launch: a grid z of nq * L
   for (int i = 0; i < L; ++i) {
     const csa2_layer& ly = layers[i];
     int32_t r = check_attn(ly.q_attn, &ly.codes, &ly.scales, s->query_pos, s->nq, s->Hq, s->D, s->K,

@@ -45,6 +45,7 @@ extern "C" int32_t csa2_topk_pool_noalloc(const int32_t* scores, int64_t ld, con
   if (!out_idx || !status || nq < 1 || n_max < 0 || n_max > (1 << 30) || k < 1 || k > 65536)
     return CSA2_ERR_INVALID_ARG;
   if (n_max > 0 && (!scores || ld < n_max)) return CSA2_ERR_INVALID_ARG;
+  if (nq > 65535) return CSA2_ERR_UNSUPPORTED;   // queries index a grid dimension
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (n_max <= kSmallMax)   // the one-CTA path keeps everything in shared memory
     return launch_topk_small(scores, ld, n_valid, cand_pos, nq, n_max, k, out_idx, out_cnt, status, st) ==

@@ -83,8 +83,10 @@ def test_rejects_bad_arguments_before_any_launch():
     # more queries than one launch's work list holds
     assert L.csa2_index_full(16, 16, ctypes.byref(keys), None, 16, 4097, 64, 128, 10, None, 0, 0, None, None,
                              0, None, None, 256, 1 << 20, 16, None) == 2
-    # top-k: k out of range
+    # top-k: k out of range; more queries than a grid dimension holds
     assert L.csa2_topk_pool(16, 10, None, None, 1, 10, 0, 16, None, None, 0, 16, None) == 1
+    assert L.csa2_topk_pool(16, 10, None, None, 65536, 10, 4, 16, None, None, 0, 16, None) == 2
+    assert L.csa2_topk_pool_noalloc(16, 10, None, None, 65536, 10, 4, 16, None, 16, None) == 2
     # reindex: K > P
     assert L.csa2_reindex(16, 16, ctypes.byref(keys), None, 16, 16, 1, 64, 128, 8, 9, 16, None, None, 256,
                           1 << 20, 16, None) == 1
@@ -131,6 +133,16 @@ def test_wait_selftest_checks_its_arguments():
     assert L.csa2_selftest_wait(0, 1000, None, 16, None) == 1                  # the barrier needs a counter
     assert L.csa2_selftest_wait(1, 1000, None, None, None) == 1                # and every kind a status word
     assert L.csa2_selftest_wait(1, 10 ** 10 + 1, None, 16, None) == 1          # limits above 10 s are refused
+
+
+def test_plan_rejects_too_many_queries_times_layers():
+    L = K.lib()
+    n = 16
+    modes = (ctypes.c_int32 * n)(*([0] + [2] * (n - 1)))
+    layers = (B.csa2_layer * n)()
+    s = B.csa2_plan_shape(nq=4096, H=64, D_idx=128, Hq=64, D=512, P=16384, K=512, window=128, max_ctx=1 << 20,
+                          softmax_scale=0.0, seq_of_query=None, query_pos=16)
+    assert L.csa2_layer_plan(modes, n, layers, ctypes.byref(s), 256, 1 << 20, 16, None) == 2
 
 
 def test_plan_rejects_reindex_first():

@@ -492,7 +492,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
 }
 
 // ------------------------------------------------------------------ FP4 cache write
-// Rows of `elem` bytes per value, 16-byte aligned: ld_x a multiple of 16 / elem.
+// fp32 or bf16 rows, each starting on 16 bytes: ld_x a multiple of the values per 16 bytes.
 static int32_t run_fp4_quantize(const void* x, bool bf16, int64_t n_rows, int32_t D, int64_t ld_x,
                                 const int32_t* dst_rows, uint8_t* codes, int64_t ld_codes, uint8_t* scales,
                                 int64_t ld_scales, int64_t n_dst_rows, int32_t* status, void* stream) {

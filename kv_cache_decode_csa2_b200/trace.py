@@ -1,6 +1,6 @@
 """Phase tracing of the kernels of one decode step (or one prefill chunk).
 
-    python -m kv_cache_decode_csa2_b200.trace [--workload decode|prefill] [--warmup W]
+    python -m kv_cache_decode_csa2_b200.trace [--workload decode|prefill] [--warmup W] [--save T.npy]
 
 Builds libcsa2_trace.so (the library with its phase markers compiled in, see
 csa2_trace_attach in include/csa2.h), sets up the bench's workload through it,
@@ -189,6 +189,7 @@ def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--workload", choices=["decode", "prefill"], default="decode")
     ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--save", default=None, help="also write the raw table (uint64 [8][1024][16][2]) to this .npy")
     args = ap.parse_args(argv)
     L = load_traced_library()
     from . import csa2 as B
@@ -221,6 +222,8 @@ def main(argv=None) -> int:
         B.check_status(s)
     B._check(L.csa2_trace_attach(None), "csa2_trace_attach")
     t = table.cpu().numpy().view(np.uint64).reshape(KERNELS, CTAS, POINTS, 2)
+    if args.save:
+        np.save(args.save, t)
     ghz = clock_ghz(t)
     print(f"workload: {args.workload}")
     print(format_report(summarize(t, ghz), ghz))

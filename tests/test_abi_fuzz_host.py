@@ -74,3 +74,26 @@ def test_random_arguments_return_documented_codes():
             assert call() in CODES
     # zero rows is the one call here with nothing to launch: it succeeds without a device
     assert L.csa2_fp4_quantize(1 << 20, 0, 512, 512, None, 1 << 20, 256, 1 << 20, 16, 16, 1 << 20, None) == 0
+
+
+def test_random_plans_return_documented_codes():
+    L = K.lib()
+    rng = random.Random(11)
+    for _ in range(300):
+        n = rng.choice([0, 1, 2, 3, 8, 16, 17])
+        size = max(n, 1)
+        modes = (ctypes.c_int32 * size)(*[rng.choice([-1, 0, 0, 1, 2, 3]) for _ in range(size)])
+        layers = (B.csa2_layer * size)()
+        for ly in layers:
+            ly.q, ly.w, ly.q_attn, ly.out = _ptr(rng), _ptr(rng), _ptr(rng), _ptr(rng)
+            ly.keys, ly.codes, ly.scales = _rows(rng), _rows(rng), _rows(rng)
+            if rng.random() < 0.3:
+                ly.local_kv = _rows(rng)
+        s = B.csa2_plan_shape(nq=_int(rng), H=_int(rng), D_idx=rng.choice([64, 128, 96]), Hq=rng.choice([8, 64, 12]),
+                              D=rng.choice([128, 512, 256]), P=_int(rng), K=_int(rng), window=_int(rng),
+                              max_ctx=_int(rng), softmax_scale=0.0, seq_of_query=_ptr(rng), query_pos=_ptr(rng),
+                              group_queries=rng.choice([0, 1]))
+        args = (modes if rng.random() < 0.95 else None, n, layers if rng.random() < 0.95 else None,
+                ctypes.byref(s) if rng.random() < 0.95 else None)
+        assert L.csa2_layer_plan(*args, _ptr(rng), _int(rng, 1 << 40), _ptr(rng), None) in CODES
+        assert L.csa2_layer_plan_workspace(args[0], n, args[3]) >= 0

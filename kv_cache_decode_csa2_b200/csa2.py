@@ -258,6 +258,8 @@ def csa2_sparse_attn_fp4(q, codes: Rows, scales: Rows, query_pos, sel_idx, out, 
         code = L.csa2_sparse_attn_fp4(_ptr(q), ctypes.byref(cr), ctypes.byref(sr), *tail)
         _check(code, "csa2_sparse_attn_fp4")
     else:
+        if local_kv.data.dtype != torch.bfloat16:
+            raise ValueError("local_kv rows must be bfloat16")
         lr = local_kv.c()
         code = L.csa2_sparse_attn_fp4_local(_ptr(q), ctypes.byref(cr), ctypes.byref(sr), ctypes.byref(lr), *tail)
         _check(code, "csa2_sparse_attn_fp4_local")
@@ -335,6 +337,8 @@ class LayerPlan:
             c.pool_idx, c.pool_cnt = _ptr(ly.pool_idx), _ptr(ly.pool_cnt)
             c.sel_idx, c.sel_cnt = _ptr(ly.sel_idx), _ptr(ly.sel_cnt)
             if ly.local_kv is not None:
+                if ly.local_kv.data.dtype != torch.bfloat16:
+                    raise ValueError(f"layer {i}: local_kv rows must be bfloat16")
                 c.local_kv = ly.local_kv.c()
         s = csa2_plan_shape()
         s.nq, s.H, s.D_idx, s.Hq, s.D, s.P, s.K = nq, H, D_idx, Hq, D, P, K

@@ -200,7 +200,7 @@ def fp4_dequant(codes: np.ndarray, scales: np.ndarray, dim: int) -> np.ndarray:
     value[j] = e2m1(code j) * e4m3(scale of block j // 32).
 
     [AD] Act 3: "FP4 main KV caching"; [YS] item 2: "KV values are compressed
-    from FP8 (8 bits) to FP4 (4 bits)".  READING 10: the nibble order and the
+    from FP8 (8 bits) to FP4 (4 bits)".  READING 9: the nibble order and the
     two-plane row layout.
     """
     codes = np.asarray(codes, dtype=np.uint8)
@@ -245,7 +245,7 @@ def fp4_quantize(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
       code  = E2M1 nearest to x/scale (ties to even, saturating at +-6)
     If the scale decodes to 0, every code in the block is 0.  A value that
     rounds to magnitude 0 is stored as +0 (code 0).
-    READING 11: the scale is rounded to nearest, so the block maximum can be
+    READING 10: the scale is rounded to nearest, so the block maximum can be
     clipped to 6*scale.  This is the cache-write side of the FP4 main KV cache
     ([AD] Act 3).
     """
@@ -387,7 +387,11 @@ def prefill_query(q, w, keys, q_attn, codes, scales, pos: int, topk: int, window
     """One query of a causal prefill chunk at position ``pos``.  Its top-k is
     taken over its whole causal prefix 0..pos (there is no pool), and it then
     attends to that top-k together with the window.
-    Returns (sel_idx, attn_set, o, lse)."""
+    Returns (sel_idx, attn_set, o, lse).
+
+    READING 14: every query of the chunk sees rows 0..pos only, for the index,
+    the window and the attention, and keeps its top-k of the whole prefix.
+    READING 7 (as for decode): the cache already holds the token at pos."""
     s = index_scores(q, w, keys[:pos + 1])
     sel = top_k_positions(s, np.arange(pos + 1, dtype=np.int64), topk)
     S = attention_set(sel, pos, window)

@@ -9,5 +9,3 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: full-size parity case")
-    config.addinivalue_line("markers", "gpu_pending: GPU parity written but not yet run on a B200; selected only "
-                                       "with -m gpu_pending, skipped without a device")

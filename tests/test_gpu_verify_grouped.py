@@ -10,7 +10,7 @@ import synth
 from kv_cache_decode_csa2_b200 import csa2 as B
 from tests import gpu_cases as G
 
-pytestmark = pytest.mark.gpu_pending   # written, not yet run on a B200
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module", autouse=True)

@@ -9,7 +9,7 @@ import torch
 
 from kv_cache_decode_csa2_b200 import csa2 as B
 
-pytestmark = pytest.mark.gpu_pending   # written, not yet run on a B200
+pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 

@@ -38,10 +38,11 @@ see tests/test_oracle_pins.py):
                       s(q) - s(-q) = keys . (sum_h w_h q_h).  The formula
                       itself is READING 1 (parity unpinned by the pages).
   top_k_positions     pinned: repeated-maximum extraction, adversarial ties.
-  e2m1_decode         pinned: OCP MX E2M1 table (tests/golden) and torch's
-                      float4_e2m1fn_x2 where torch can convert it.
+  e2m1_decode         pinned: OCP MX E2M1 table (tests/golden) and
+                      ml_dtypes' float4_e2m1fn decoder on all 16 codes.
   e4m3_decode         pinned: torch.float8_e4m3fn on all 256 bytes, OFP8 table.
-  fp4_quantize        pinned: exhaustive nearest-code search, round trips.
+  fp4_quantize        pinned: exhaustive nearest-code search, round trips,
+                      ml_dtypes' float -> float4_e2m1fn rounding inside the range.
   sparse_attention    pinned: torch scaled_dot_product_attention (fp64) when
                       the set is the whole context; closed forms.
   decode_layer_plan   pinned: separate pure-Python brute force on tiny inputs.

@@ -132,6 +132,39 @@ def test_e2m1_matches_ocp_table():
     assert np.array_equal(np.signbit(got), np.signbit(want))
 
 
+def test_e2m1_all_codes_match_ml_dtypes():
+    """A second, independent decoder of OCP E2M1: ml_dtypes.float4_e2m1fn
+    (one code per byte, in the low nibble)."""
+    ml = pytest.importorskip("ml_dtypes")
+    want = np.arange(16, dtype=np.uint8).view(ml.float4_e2m1fn).astype(np.float64)
+    got = O.e2m1_decode(np.arange(16))
+    assert np.array_equal(got, want)
+    assert np.array_equal(np.signbit(got), np.signbit(want))
+
+
+def test_e2m1_rounding_matches_ml_dtypes_in_range():
+    """Inside the E2M1 range the quantiser's code choice is round to nearest,
+    ties to even: on a grid that holds every representable value, every
+    midpoint between neighbours and points just beside them, the magnitude
+    it stores equals ml_dtypes' float -> float4_e2m1fn conversion (scale 1)."""
+    ml = pytest.importorskip("ml_dtypes")
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    mids = (mags[:-1] + mags[1:]) / 2
+    pts = np.unique(np.concatenate([mags, mids, mids - 1e-6, mids + 1e-6, np.linspace(0, 6, 241)]))
+    x = np.concatenate([pts, -pts])
+    # one block per value: the block maximum 6 fixes the scale at exactly 1.0 (E4M3 0x38)
+    blocks = np.zeros((len(x), 32))
+    blocks[:, 0] = x
+    blocks[:, 1] = 6.0
+    codes, scales = O.fp4_quantize(blocks)
+    assert (scales == 0x38).all()
+    got = O.e2m1_decode(codes[:, 0] & 0xF)
+    want = x.astype(np.float32).astype(ml.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(np.abs(got), np.abs(want))
+    nz = want != 0
+    assert np.array_equal(np.sign(got[nz]), np.sign(want[nz]))
+
+
 def test_e4m3_all_bytes_match_torch():
     b = torch.arange(256, dtype=torch.int32).to(torch.uint8)
     want = b.view(torch.float8_e4m3fn).to(torch.float64).numpy()

@@ -47,6 +47,8 @@ see tests/test_oracle_pins.py):
                       the set is the whole context; closed forms.
   decode_layer_plan   pinned: separate pure-Python brute force on tiny inputs.
   prefill_query       pinned: equals decode at the same position (property).
+  attention_combine   pinned: equals sparse_attention over the union on random
+                      partitions (one set empty), and the single-set identity.
   kv_rows_local_window  pinned: closed forms (one window row, uniform
                       softmax over ring slots and FP4 rows), the separate
                       brute force of the plan with local rings, and equality
@@ -290,6 +292,33 @@ def sparse_attention(q: np.ndarray, kv_rows: np.ndarray, softmax_scale: float | 
     l = p.sum(axis=1, keepdims=True)
     o = (p @ kv) / l
     return o, (mx + np.log(l))[:, 0]
+
+
+def attention_combine(outs, lses):
+    """Attention over the union of disjoint row sets, from the result of each
+    set.
+
+    outs float [R][Hq][D] and lses float [R][Hq] are sparse_attention's
+    (o, lse) over R disjoint sets of rows; an empty set has lse = -inf (its o
+    is ignored).  Softmax over the union is each set's softmax scaled by that
+    set's share of the total mass:
+      LSE = log sum_r exp(lse_r),   o = sum_r exp(lse_r - LSE) o_r.
+    Returns (o float64 [Hq][D], LSE float64 [Hq]).  A head whose sets are all
+    empty gets o = 0 and LSE = -inf.
+    READING 16: a context split over several GPUs attends slice by slice and
+    combines the slices' results.  The pages scale context by selection
+    ([AD] Act 2) and do not say how a sharded context is attended.
+    """
+    outs = np.asarray(outs, dtype=np.float64)
+    lses = np.asarray(lses, dtype=np.float64)
+    M = lses.max(axis=0)                                            # [Hq]
+    some = np.isfinite(M)
+    w = np.where(np.isfinite(lses), np.exp(lses - np.where(some, M, 0.0)), 0.0)   # [R][Hq]
+    L = w.sum(axis=0)
+    safe = np.where(L > 0, L, 1.0)
+    outs = np.where(np.isfinite(lses)[:, :, None], outs, 0.0)      # an empty set's o is not used
+    o = np.einsum("rh,rhd->hd", w, outs) / safe[:, None]
+    return np.where(some[:, None], o, 0.0), np.where(some, M + np.log(safe), -np.inf)
 
 
 # =============================================================== the layer's local window cache

@@ -455,3 +455,39 @@ def test_local_window_needs_a_ring_as_long_as_the_window():
 def test_plan_rejects_bad_first_mode():
     with pytest.raises(ValueError):
         O.decode_layer_plan([1, 0], [{}, {}], 0, 4, 2, 2)
+
+
+# ------------------------------------------------------------------ combine of partial attention
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_attention_combine_equals_attention_over_the_union(seed):
+    """Softmax attention over a set of rows equals the combine of attention
+    over any partition of it (one part left empty): the identity the
+    context-sharded decode rests on, checked in fp64."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((8, 64))
+    kv = rng.standard_normal((300, 64)) * 2.0
+    parts = rng.integers(0, 3, size=300)          # part 3 stays empty
+    outs, lses = [], []
+    for r in range(4):
+        rows = kv[parts == r]
+        if len(rows):
+            o, l = O.sparse_attention(q, rows)
+        else:
+            o, l = np.full((8, 64), np.nan), np.full(8, -np.inf)
+        outs.append(o)
+        lses.append(l)
+    got_o, got_l = O.attention_combine(outs, lses)
+    want_o, want_l = O.sparse_attention(q, kv)
+    assert np.allclose(got_o, want_o, rtol=1e-12, atol=1e-12)
+    assert np.allclose(got_l, want_l, rtol=1e-12, atol=1e-12)
+
+
+def test_attention_combine_single_part_and_all_empty():
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((4, 32))
+    kv = rng.standard_normal((50, 32))
+    o, l = O.sparse_attention(q, kv)
+    got_o, got_l = O.attention_combine([o], [l])
+    assert np.array_equal(got_o, o) and np.allclose(got_l, l, rtol=0, atol=1e-15)
+    e_o, e_l = O.attention_combine([np.ones((4, 32)), np.ones((4, 32))], [np.full(4, -np.inf)] * 2)
+    assert (e_o == 0).all() and np.isneginf(e_l).all()

@@ -1,37 +1,47 @@
-"""Benchmark of the CSA2 decode step: the 1M-token-context, 8-layer plan
-[full, reindex, reuse, reuse, reindex, reuse, reuse, reuse].
+"""Benchmark of the CSA2 sparse-attention decode path on one B200 (or N, one
+process per GPU).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference] [--workload NAME]
 
-A step is one pass of the whole hot path over one decode query:
-  - full-mode index scoring of all 1,048,576 positions;
-  - the 16,384-candidate pool and the layer's top-512;
-  - two reindex layers over the pool;
-  - FP4 sparse attention (512 selected + 128 window positions) in all 8 layers.
-The step runs as one csa2_layer_plan call, captured once into a CUDA graph
-per input replica.  Inputs are synthetic (seeded, see synth/), resident in
-HBM, and rotate over 4 device replicas of the whole state: about 141 MB read
-per step, 564 MB per cycle against a 126 MB L2.  With N GPUs every rank
-decodes its own sequence: weak scaling, no data-path collective.  Rank 0
-prints one JSON line.
+Workloads (--workload):
+  decode    (default) the 1M-token-context 8-layer step: plan [full, reindex,
+            reuse, reuse, reindex, reuse, reuse, reuse], pool 16,384, top-512
+            + 128-token window, int8 indexer 64x128, FP4 KV d512, 64 query heads.
+  tiny      the same path at context 4096 with the small shapes (indexer 4x64,
+            pool 1024, top-64, 8 query heads, KV d128), one full layer.
+  single    one full layer at context 131,072 with the 1M step's shapes.
+  ragged    32 sequences of 32K-262K rows in 64-row pages (shuffled page
+            table), one full layer each: queries/s.
+  verify    a speculative-verify block of 5 causal queries at the end of the
+            1M context, all 8 layers, the index scan shared by the block.
+  prefill   2048 causal queries at positions 260096-262143 of a 262,144-row
+            context: int8 index GEMM, per-query top-512 over the prefix,
+            attention.  queries/s and the index stage's int8 TOP/s.
+  quantize  the FP4 cache write of 1,048,576 bf16 rows of d512.
 
---impl reference times the CPU oracle (oracle/) on the same workload, on this
-host's cores; there is no other reference implementation of this path.
+A step is one pass of the whole hot path over one batch of synthetic input,
+through the library's C ABI (csa2_layer_plan for the decode workloads),
+captured once per input replica in a CUDA graph.  Inputs are seeded (synth/),
+resident in HBM, and rotate over device replicas whose caches together exceed
+the L2, so no step reads another step's data from L2.  The JSON line gives:
+  value       units per second (median of 5 repeats of exactly --steps
+              timed steps, each repeat bracketed by a barrier and a device
+              synchronisation, max over ranks);
+  steps100    the same with at least 100 replays per repeat;
+  hbm         algorithmic bytes per step, GB/s and fractions of 8 TB/s and of
+              the measured copy peak;
+  roofline    the dominant kernel alone (the index-score stream), its
+              algorithmic bytes per launch over its CUDA-event time;
+  e2e         the same metric through the C ABI with host buffers: one pinned
+              host-to-device copy of the step's inputs, the plan call, one
+              device-to-host copy of its outputs, every step;
+  cpu_baseline  the CPU oracle (oracle/) on this host's cores, on a bounded
+              sample of the same workload.
+With N GPUs every rank runs its own copy of the workload: weak scaling, no
+data-path collective.  Rank 0 prints one JSON line.
 
-    python bench.py --workload prefill [--steps K] [--warmup W]
-
-times the prefill-chunk configuration instead: 2048 causal queries at
-positions 260096-262143 of a 262,144-row context, each scoring its whole
-prefix with the int8 indexer, keeping its top-512 and attending to them plus
-the 128-row window (one csa2_index_full and one csa2_sparse_attn_fp4 call,
-captured in a CUDA graph per replica).  It prints queries/s and the int8
-TOP/s of the index stage.
-
-    python bench.py --workload quantize [--steps K] [--warmup W]
-
-times the FP4 cache write: 1,048,576 bf16 rows of d512 (one layer's latent KV
-at the 1M context) stored as E2M1 codes and E4M3 scales by
-csa2_fp4_quantize, in rows/s and HBM GB/s.
+--impl reference times the CPU oracle on the same workload on this host's
+cores; there is no other implementation of this path to compare against.
 """
 from __future__ import annotations
 
@@ -55,17 +65,31 @@ import synth  # noqa: E402
 
 METRIC = "decode steps/s and HBM GB/s (% of B200 roofline) at 1M-token context"
 WL = synth.C2_1M_PLAN
+WL_VERIFY = synth.scaled(synth.C2_1M_PLAN, name="verify_5q_ctx1048576_8layer",
+                         prefill=(5, int(synth.C2_1M_PLAN.lengths()[0]) - 5))
+# name: (workload, metric, unit, units per step, group the queries of a sequence)
+DECODE_WORKLOADS = {
+    "decode": (WL, METRIC, "steps/s", 1, False),
+    "tiny": (synth.C0_TINY, "decode steps/s and us per step at 4096-token context (small shapes)", "steps/s", 1,
+             False),
+    "single": (synth.C1_SINGLE, "decode steps/s and HBM GB/s at 131072-token context", "steps/s", 1, False),
+    "ragged": (synth.C3_RAGGED, "decode queries/s and HBM GB/s over 32 paged ragged sequences (32K-262K rows)",
+               "queries/s", 32, False),
+    "verify": (WL_VERIFY, "verify blocks/s (5 queries sharing one index scan) at 1M-token context",
+               "blocks/s", 1, True),
+}
 METRIC_PREFILL = "prefill-chunk queries/s and index int8 TOP/s (2048 causal queries, 262144 context)"
 WL_PREFILL = synth.C4_PREFILL
 METRIC_QUANT = "FP4 cache write rows/s and HBM GB/s (1,048,576 bf16 rows of d512 -> E2M1 + E4M3)"
-QUANT_SAMPLE_ROWS = 16384
-# DRAM bytes (read + write) of one index-score launch on the decode workload,
-# from one ncu capture of this kernel on it (its summary is kept with the
-# profiles); to be reset to None whenever that kernel changes.
-K1_TRAFFIC_BYTES = 134_273_792 + 4_593_664
-N_REPLICAS = 4
+QUANT_SAMPLE_ROWS = 65536
+# DRAM bytes (read + write) of one index-score launch on the 1M decode
+# workload, from one ncu capture of this kernel (its summary is kept with the
+# profiles); None when that kernel changed after the capture.
+K1_TRAFFIC_BYTES = {"decode": 134_273_792 + 4_593_664}
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 NOMINAL_HBM_GBS = 8000.0
+REPEATS = 5
+MAX_REPLICAS = 256
 
 
 def peaks() -> dict:
@@ -77,6 +101,24 @@ def peaks() -> dict:
         return {"hbm_gbs": 6650.0, "src": "fallback"}
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
 def device_facts(dev) -> dict:
     """The device's L2 size, and a read-only HBM stream rate measured here:
     torch.sum over 2 GiB of fp32 (larger than L2), best of 5 after one warm-up,
@@ -85,10 +127,7 @@ def device_facts(dev) -> dict:
     out = {"l2_bytes": None, "read_only_gbs": None, "read_only_how": "torch.sum of 2 GiB fp32, best of 5"}
     if getattr(dev, "type", None) != "cuda":
         return out
-    try:
-        out["l2_bytes"] = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0)) or None
-    except Exception:
-        pass
+    out["l2_bytes"] = l2_bytes(dev)
     try:
         x = torch.ones(1 << 29, dtype=torch.float32, device=dev)
         best = None
@@ -107,6 +146,13 @@ def device_facts(dev) -> dict:
     except Exception:
         pass
     return out
+
+
+def l2_bytes(dev) -> int:
+    try:
+        return int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0)) or (126 << 20)
+    except Exception:
+        return 126 << 20
 
 
 # ----------------------------------------------------------------- distributed plumbing
@@ -202,281 +248,296 @@ def gpu_id(dev) -> str:
         return str(dev.index or 0)
 
 
-# ----------------------------------------------------------------- device state of one replica
-def host_inputs(wl):
-    """Host arrays of one decode step (everything except the FP4 KV values)."""
-    lens = wl.lengths()
-    pos = int(lens[0]) - 1
-    layers = []
-    for l, mode in enumerate(wl.modes):
-        d = {"q_attn": synth.attn_query(wl, l, 0)}
-        if mode != synth.REUSE:
-            d["keys"] = synth.index_keys(wl, l, 0)
-            d["q"], d["w"] = synth.index_query(wl, l, 0)
-        layers.append(d)
-    return pos, layers
+# ----------------------------------------------------------------- timing
+def time_replays(graphs, n: int, stream, world: int, dev) -> float:
+    """Milliseconds per replay over exactly n replays (rotating over the
+    graphs), bracketed by a barrier and a device synchronisation on both
+    sides; the max over ranks."""
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        a.record(stream)
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    return max_over_ranks(a.elapsed_time(b), world, dev) / n
 
 
-def build_device_state(wl, host, dev, status):
-    from kv_cache_decode_csa2_b200 import csa2 as B
-    pos, hl = host
-    n = pos + 1
-    layers = []
-    for l, mode in enumerate(wl.modes):
-        d = hl[l]
-        codes = torch.empty((n, wl.attn_dim // 2), dtype=torch.uint8, device=dev)
-        scales = torch.empty((n, wl.attn_dim // 32), dtype=torch.uint8, device=dev)
-        step = 1 << 17
-        for a in range(0, n, step):            # FP4 cache written by the library's quantiser
-            b = min(n, a + step)
-            x = torch.from_numpy(synth.kv_values(wl, l, 0, a, b)).to(dev, non_blocking=False)
-            B.csa2_fp4_quantize(x, codes[a:b], scales[a:b], status=status)
-        ly = B.Layer(q_attn=torch.from_numpy(d["q_attn"]).to(dev).to(torch.bfloat16)[None].contiguous(),
-                     codes=B.Rows(codes), scales=B.Rows(scales),
-                     out=torch.empty((1, wl.attn_heads, wl.attn_dim), dtype=torch.bfloat16, device=dev),
-                     lse=None)
-        if mode != synth.REUSE:
-            ly.keys = B.Rows(torch.from_numpy(d["keys"]).to(dev))
-            ly.q = torch.from_numpy(d["q"]).to(dev)[None].contiguous()
-            ly.w = torch.from_numpy(d["w"]).to(dev)[None].contiguous()
-            ly.sel_idx = torch.empty((1, wl.topk), dtype=torch.int32, device=dev)
-            ly.sel_cnt = torch.empty((1,), dtype=torch.int32, device=dev)
-        if mode == synth.FULL:
-            ly.pool_idx = torch.empty((1, wl.pool), dtype=torch.int32, device=dev)
-            ly.pool_cnt = torch.empty((1,), dtype=torch.int32, device=dev)
-        layers.append(ly)
-    return layers
+def timed_block(graphs, steps: int, stream, world: int, dev) -> dict:
+    """REPEATS repeats of exactly `steps` replays, then REPEATS repeats of at
+    least 100 replays: per-step milliseconds of each repeat and the medians."""
+    per = [time_replays(graphs, steps, stream, world, dev) for _ in range(REPEATS)]
+    n100 = max(100, steps)
+    per100 = [time_replays(graphs, n100, stream, world, dev) for _ in range(REPEATS)]
+    return {"ms": statistics.median(per), "ms_all": per, "ms100": statistics.median(per100), "ms100_all": per100,
+            "replays100": n100}
 
 
-def clone_layers(layers, dev):
-    from kv_cache_decode_csa2_b200 import csa2 as B
-    out = []
-    for ly in layers:
-        c = B.Layer(q_attn=ly.q_attn.clone(), codes=B.Rows(ly.codes.data.clone()),
-                    scales=B.Rows(ly.scales.data.clone()), out=torch.empty_like(ly.out))
-        if ly.keys is not None:
-            c.keys = B.Rows(ly.keys.data.clone())
-            c.q, c.w = ly.q.clone(), ly.w.clone()
-            c.sel_idx, c.sel_cnt = torch.empty_like(ly.sel_idx), torch.empty_like(ly.sel_cnt)
-        if ly.pool_idx is not None:
-            c.pool_idx, c.pool_cnt = torch.empty_like(ly.pool_idx), torch.empty_like(ly.pool_cnt)
-        out.append(c)
-    return out
+def load_for(graphs, seconds: float, stream):
+    """Untimed replays for about `seconds`, so the clock samples see the GPU
+    under this load before the timed repeats."""
+    t0 = time.time()
+    i = 0
+    while time.time() - t0 < seconds:
+        with torch.cuda.stream(stream):
+            for _ in range(32):
+                graphs[i % len(graphs)].replay()
+                i += 1
+        torch.cuda.synchronize()
 
 
-def algorithmic_bytes(wl, layers, pos) -> tuple[int, dict]:
-    """Bytes the method must move per step: the full layer's key rows, the pool
-    rows each reindex layer gathers, the FP4 rows of every layer's attention
-    set, queries, head weights and outputs.  Scores, histograms and index lists
-    are intermediates and are not counted."""
-    ctx = pos + 1
-    row_idx = wl.idx_dim
-    row_fp4 = wl.attn_dim // 2 + wl.attn_dim // 32
-    wstart = max(0, pos - wl.window + 1)
-    parts = {"full_keys": ctx * row_idx, "reindex_gather": 0, "attn_rows": 0, "q_w_out": 0}
-    sel = None
-    for l, mode in enumerate(wl.modes):
-        ly = layers[l]
-        if mode != synth.REUSE:
-            sel = ly.sel_idx[0, :int(ly.sel_cnt[0])].cpu().numpy()
-            parts["q_w_out"] += wl.idx_heads * wl.idx_dim + wl.idx_heads
-        if mode == synth.REINDEX:
-            parts["reindex_gather"] += int(layers[0].pool_cnt[0]) * row_idx
-        n_s = int((sel < wstart).sum()) + (pos - wstart + 1)
-        parts["attn_rows"] += n_s * row_fp4
-        parts["q_w_out"] += 2 * wl.attn_heads * wl.attn_dim * 2
-    return sum(parts.values()), parts
+def kernels_in(fn, stream) -> int | None:
+    """How many of the library's kernels one call of fn launches, counted by
+    torch's profiler (CUPTI) outside the timed region; None if unavailable."""
+    try:
+        from torch.profiler import ProfilerActivity, profile
+        torch.cuda.synchronize()
+        with profile(activities=[ProfilerActivity.CUDA]) as prof:
+            with torch.cuda.stream(stream):
+                fn()
+            torch.cuda.synchronize()
+        n = 0
+        for ev in prof.events():
+            if getattr(ev, "device_type", None) is not None and "csa2" in ev.name and "Memset" not in ev.name:
+                if str(ev.device_type).endswith("CUDA"):
+                    n += 1
+        return n or None
+    except Exception:
+        return None
 
 
-def kernels_per_step(wl) -> int:
-    """Kernels one plan step launches on this workload: one launch that zeroes
-    the step's scratch, the index-score stream and the pool select of the full
-    layer, one fused scoring + top-k launch for the reindex layers of the pool,
-    and one attention launch for all layers (the ncu launch list in profiles/
-    shows the same five per step)."""
-    n_re = sum(1 for m in wl.modes if m == synth.REINDEX)
-    n_full = sum(1 for m in wl.modes if m == synth.FULL)
-    return 1 + 2 * n_full + (1 if n_re else 0) + 1
+# ----------------------------------------------------------------- the CPU oracle
+class OracleQuery:
+    """One query of a decode workload through the CPU oracle: every layer of
+    the plan (full index, pool and selection; reindex; reuse; attention).
 
+    Every step function is the oracle's own (oracle/); this class sequences
+    them the way decode_layer_plan does and times them.  The full layer's scan
+    of every key row can run on T host threads, each scoring a contiguous
+    slice of the rows with the oracle's index_scores; BLAS gets T threads.
+    The FP4 rows of each layer's attention set are stored by the oracle's
+    quantiser before the timed run (the cache write is not part of a step)."""
 
-# ----------------------------------------------------------------- the CPU oracle baseline
-class OracleStep:
-    """One decode step of the CPU oracle on this workload, on one host core.
-
-    Every step function is the oracle's own (oracle/).  This class only
-    sequences them the way decode_layer_plan does, so that the context-linear
-    part (the full layer's scan of every key row) can be timed on a 1/f slice
-    of the positions and scaled by f.  The pool top-k, reindex and attention
-    always run in full, over the full layer's real scores (computed once,
-    untimed).  With f = 1 a step is exactly one whole oracle decode step."""
-
-    def __init__(self, wl, host):
+    def __init__(self, wl, query: int):
         import oracle as O
         self.O, self.wl = O, wl
-        self.pos, self.hl = host
+        sq, qp = wl.query_positions()
+        self.seq, self.pos = int(sq[query]), int(qp[query])
         n = self.pos + 1
-        full = self.hl[0]
-        self.scores0 = O.index_scores(full["q"], full["w"], full["keys"][:n])
+        self.layers = []
+        for l, mode in enumerate(wl.modes):
+            d = {"q_attn": synth.attn_query(wl, l, query)}
+            if mode != synth.REUSE:
+                d["keys"] = synth.index_keys(wl, l, self.seq, 0, n)
+                d["q"], d["w"] = synth.index_query(wl, l, query)
+            self.layers.append(d)
         self.codes = []
         pool = sel = None
-        for l, mode in enumerate(wl.modes):          # FP4 rows the step reads, stored by the oracle
-            d = self.hl[l]
+        scores0 = O.index_scores(self.layers[0]["q"], self.layers[0]["w"], self.layers[0]["keys"])
+        for l, mode in enumerate(wl.modes):                 # FP4 rows the step reads (untimed)
+            d = self.layers[l]
             if mode == synth.FULL:
-                pool = O.top_k_positions(self.scores0, np.arange(n), wl.pool)
-                sel = O.top_k_positions(self.scores0[pool], pool, wl.topk)
+                pool = O.top_k_positions(scores0, np.arange(n), wl.pool)
+                sel = O.top_k_positions(scores0[pool], pool, wl.topk)
             elif mode == synth.REINDEX:
                 _, sel = O.reindex(d["q"], d["w"], d["keys"], pool, wl.topk)
             S = O.attention_set(sel, self.pos, wl.window)
             codes = np.zeros((n, wl.attn_dim // 2), np.uint8)
             scales = np.zeros((n, wl.attn_dim // 32), np.uint8)
-            x = np.concatenate([synth.kv_values(wl, l, 0, int(r), int(r) + 1) for r in S])
+            x = np.concatenate([synth.kv_values(wl, l, self.seq, int(r), int(r) + 1) for r in S])
             codes[S], scales[S] = O.fp4_quantize(x)
             self.codes.append((codes, scales))
 
-    def run(self, f: int = 1, slice_i: int = 0) -> tuple[float, float]:
-        """Returns (seconds of the step, seconds of the scaled scan part)."""
+    def _scores(self, d, threads: int, lo: int, hi: int):
+        O = self.O
+        if threads <= 1:
+            return O.index_scores(d["q"], d["w"], d["keys"][lo:hi])
+        from concurrent.futures import ThreadPoolExecutor
+        cuts = [lo + (hi - lo) * i // threads for i in range(threads + 1)]
+        with ThreadPoolExecutor(threads) as ex:
+            parts = list(ex.map(lambda i: O.index_scores(d["q"], d["w"], d["keys"][cuts[i]:cuts[i + 1]]),
+                                range(threads)))
+        return np.concatenate(parts)
+
+    def run(self, threads: int = 1, f: int = 1, slice_i: int = 0) -> float:
+        """Seconds of one query.  With f > 1 the full layer's scan is timed
+        on slice slice_i of f equal slices of the rows and scaled by f (its
+        pool and selection then use the full scores, computed untimed)."""
         from threadpoolctl import threadpool_limits
         O, wl, pos = self.O, self.wl, self.pos
         n = pos + 1
-        with threadpool_limits(1):
-            full = self.hl[0]
-            lo = (n * slice_i) // f
-            hi = (n * (slice_i + 1)) // f
-            t0 = time.perf_counter()
-            O.index_scores(full["q"], full["w"], full["keys"][lo:hi])
-            t_scan = (time.perf_counter() - t0) * f
-            t1 = time.perf_counter()
+        t_total = 0.0
+        with threadpool_limits(threads):
             pool = sel = None
             for l, mode in enumerate(wl.modes):
-                d = self.hl[l]
+                d = self.layers[l]
+                t0 = time.perf_counter()
                 if mode == synth.FULL:
-                    pool = O.top_k_positions(self.scores0, np.arange(n), wl.pool)
-                    sel = O.top_k_positions(self.scores0[pool], pool, wl.topk)
+                    if f > 1:
+                        lo, hi = n * slice_i // f, n * (slice_i + 1) // f
+                        self._scores(d, threads, lo, hi)
+                        t_total += (time.perf_counter() - t0) * f
+                        s = self._scores(d, threads, 0, n)
+                        t0 = time.perf_counter()
+                    else:
+                        s = self._scores(d, threads, 0, n)
+                    pool = O.top_k_positions(s, np.arange(n), wl.pool)
+                    sel = O.top_k_positions(s[pool], pool, wl.topk)
                 elif mode == synth.REINDEX:
                     _, sel = O.reindex(d["q"], d["w"], d["keys"], pool, wl.topk)
                 S = O.attention_set(sel, pos, wl.window)
                 codes, scales = self.codes[l]
                 O.sparse_attention(d["q_attn"], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
-            t_rest = time.perf_counter() - t1
-        return t_scan + t_rest, t_scan
+                t_total += time.perf_counter() - t0
+        return t_total
 
 
-def cpu_cores_used() -> int:
-    # the timed oracle runs with BLAS limited to one thread; numpy's int64
-    # matrix product and its sorts are single-threaded anyway
-    return 1
+def oracle_sample(key: str):
+    """(OracleQuery, queries of a step it stands for, description) of a
+    decode workload's bounded CPU sample."""
+    wl, _, _, units, _ = DECODE_WORKLOADS[key]
+    sq, qp = wl.query_positions()
+    if key == "ragged":
+        q = 0
+        return OracleQuery(wl, q), 1, f"query 0 of the 32 (sequence 0, {int(qp[q]) + 1} rows), scaled to queries/s"
+    if key == "verify":
+        q = len(qp) - 1
+        return OracleQuery(wl, q), len(qp), "the block's last query (whole 1M prefix) through all 8 layers, x5 per block"
+    return OracleQuery(wl, 0), 1, f"one whole {len(wl.modes)}-layer decode step of the same workload"
 
 
-# ----------------------------------------------------------------- arms
+def cpu_baseline_decode(key: str, budget_s: float = 60.0) -> dict:
+    oq, per_unit, sample = oracle_sample(key)
+    cores = host_cores()
+    t_all = oq.run(cores)
+    out = {"value": 1.0 / (t_all * per_unit), "unit": DECODE_WORKLOADS[key][2], "cores": cores, "kind": "oracle",
+           "sample": sample, "cpu_model": cpu_model(),
+           "how": "full layer's key scan split over the host threads (oracle index_scores per slice), BLAS on "
+                  "the same threads; everything else single-threaded numpy"}
+    if key in ("tiny", "single"):
+        t1 = oq.run(1)
+        out["value_1core"] = 1.0 / (t1 * per_unit)
+    return out
+
+
+# ----------------------------------------------------------------- reference arm (the oracle)
 def run_reference(args, rank, world):
     if rank != 0:
         return
-    wl = WL
-    step = OracleStep(wl, host_inputs(wl))
-    # size the per-step sample so that warm-up + timed steps stay near 3 minutes
-    probe_f = 64
-    t_probe, t_scan_probe = step.run(probe_f, 0)
-    t_rest = t_probe - t_scan_probe
-    budget = 180.0 / (args.steps + args.warmup)
+    key = args.workload
+    if key == "prefill":
+        return run_reference_prefill(args)
+    if key == "quantize":
+        return run_reference_quantize(args)
+    wl, metric, unit, units, _ = DECODE_WORKLOADS[key]
+    oq, per_unit, sample = oracle_sample(key)
+    cores = host_cores()
+    t = oq.run(cores)
+    budget = 180.0 / (args.steps + args.warmup)   # warm-up + timed steps near 3 minutes
     f = 1
-    while t_scan_probe / f + t_rest > budget and f < 1024:
+    while t / f > budget and f < 1024 and wl.lengths().max() > 16384:
         f *= 2
     for i in range(args.warmup):
-        step.run(f, i % f)
-    ts = [step.run(f, i % f)[0] for i in range(args.steps)]
-    sec = sum(ts) / len(ts)
+        oq.run(cores, f, i % f)
+    ts = [oq.run(cores, f, i % f) * per_unit for i in range(args.steps)]
+    sec = statistics.median(ts)
     v = 1.0 / sec
-    sample = ("whole 8-layer decode steps of the 1M-context workload" if f == 1 else
-              f"8-layer decode steps of the 1M-context workload; the full layer's scan timed on 1/{f} of "
-              f"the key rows (rotating) and scaled by {f}, everything else in full")
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+    if f > 1:
+        sample += f"; the full layer's scan timed on 1/{f} of the key rows (rotating) and scaled by {f}"
+    line = {"impl": "reference", "metric": metric, "value": v, "unit": unit, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int64,f64", "data": "synthetic",
-            "config": config_dict(wl),
-            "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cpu_cores_used(), "kind": "oracle",
-                             "sample": sample},
-            "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": config_dict(key, wl),
+            "cpu_baseline": {"value": v, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample,
+                             "cpu_model": cpu_model()},
+            "e2e": {"value": v, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
-def config_dict(wl) -> dict:
-    return {"workload": wl.name, "ctx": int(wl.lengths()[0]), "batch": 1,
-            "layer_plan": ",".join(synth.MODE_NAMES[m] for m in wl.modes), "pool": wl.pool, "topk": wl.topk,
-            "window": wl.window, "indexer": f"int8 {wl.idx_heads}x{wl.idx_dim}, w int8",
-            "kv": f"FP4 E2M1 d{wl.attn_dim}, E4M3 per 32", "q_heads": wl.attn_heads,
-            "l2": f"inputs rotate over {N_REPLICAS} device replicas (~141 MB read per step, > L2 per cycle)",
-            "parallelism": "one sequence per rank"}
+def config_dict(key: str, wl, n_rep: int | None = None, rep_bytes: int | None = None) -> dict:
+    lens = wl.lengths()
+    sq, qp = wl.query_positions()
+    d = {"workload": wl.name, "ctx": int(lens.max()), "batch": len(lens), "queries": len(qp),
+         "layer_plan": ",".join(synth.MODE_NAMES[m] for m in wl.modes), "pool": wl.pool, "topk": wl.topk,
+         "window": wl.window, "indexer": f"int8 {wl.idx_heads}x{wl.idx_dim}, w int8",
+         "kv": f"FP4 E2M1 d{wl.attn_dim}, E4M3 per 32", "q_heads": wl.attn_heads,
+         "parallelism": "one workload per rank"}
+    if wl.page_rows:
+        d["paged"] = f"{wl.page_rows}-row pages, shuffled page table; lengths {int(lens.min())}..{int(lens.max())}, " \
+                     f"sum {int(lens.sum())}"
+    if key == "verify":
+        d["verify_block"] = f"{len(qp)} causal queries at positions {int(qp[0])}..{int(qp[-1])}, one sequence, " \
+                            "index scan shared (group_queries)"
+    if n_rep is not None:
+        d["l2"] = (f"inputs rotate over {n_rep} device replicas ({rep_bytes * n_rep / 1e6:.0f} MB of caches, "
+                   f"> L2)")
+    return d
 
 
-def run_gpu(args, rank, world, local):
+# ----------------------------------------------------------------- decode workloads
+def run_decode(args, rank, world, local):
     from kv_cache_decode_csa2_b200 import csa2 as B
+    from kv_cache_decode_csa2_b200 import workloads as W
+    key = args.workload
+    wl, metric, unit, units, group = DECODE_WORKLOADS[key]
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
-    wl = WL
     t_setup = time.time()
-    host = host_inputs(wl)
-    pos = host[0]
     status = B.new_status(dev)
-    base = build_device_state(wl, host, dev, status)
-    n_rep = max(1, args.replicas)
-    replicas = [base] + [clone_layers(base, dev) for _ in range(n_rep - 1)]
-    pos_dev = torch.tensor([pos], dtype=torch.int32, device=dev)
-    plans = [B.LayerPlan(list(wl.modes), r, query_pos=pos_dev, max_ctx=pos + 1, P=wl.pool, K=wl.topk,
-                         window=wl.window) for r in replicas]
+    base = W.build_decode(wl, dev, status)
+    rep_bytes = W.state_bytes(base)
+    n_rep = args.replicas or max(4, min(MAX_REPLICAS, math.ceil(2 * l2_bytes(dev) / max(rep_bytes, 1))))
+    replicas = [base] + [W.clone_decode(base, dev) for _ in range(n_rep - 1)]
+    plans = [W.decode_plan(r, group) for r in replicas]
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for p in plans:                       # ordinary calls first (one-time kernel set-up)
-            p.run()
+            p.run(stream)
     torch.cuda.synchronize()
     B.check_status(status)
     for p in plans:
         B.check_status(p.status)
-    alg_bytes, parts = algorithmic_bytes(wl, replicas[0], pos)
-
+    alg_bytes, parts = W.algorithmic_bytes(replicas[0])
+    n_kernels = kernels_in(lambda: plans[0].run(stream), stream)
     graphs = []
     for p in plans:
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            p.run()
+            p.run(stream)
         graphs.append(g)
     torch.cuda.synchronize()
     setup_s = time.time() - t_setup
 
-    # ---- timed steps (graph replays)
+    # ---- timed steps
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
             graphs[i % n_rep].replay()
     torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id(dev)) as clk:
-        time.sleep(0.3)
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for i in range(args.steps):
-                graphs[i % n_rep].replay()
-            ev1.record(stream)
-        torch.cuda.synchronize()
-    ms = ev0.elapsed_time(ev1)
-    barrier(world)
-    ms = max_over_ranks(ms, world, dev)
-    ms_step = ms / args.steps
-    value = world * args.steps / (ms / 1e3)
+        load_for(graphs, 0.4, stream)
+        tb = timed_block(graphs, args.steps, stream, world, dev)
+    ms_step = tb["ms"]
+    value = world * units / (ms_step / 1e3)
     for p in plans:
         B.check_status(p.status)
 
-    # ---- dominant kernel alone: the index-score stream over 1M keys.  Its
-    # launches (rotating over the replicas) are captured in a CUDA graph, so
-    # the CUDA events bracket kernel time, not Python launch overhead.
-    f = [r[0] for r in replicas]
-    wss = [torch.empty(B.lib().csa2_index_full_workspace(1, pos + 1, 0, 0), dtype=torch.uint8, device=dev)
-           for _ in f]
-    k_per_graph = 4 * n_rep
+    # ---- dominant kernel alone: the full layer's index-score stream (scores
+    # only), launches rotating over the replicas, captured in a CUDA graph
+    f = [r.layers[0] for r in replicas]
+    nq = len(base.query_pos)
+    ws = [torch.empty(B.lib().csa2_index_full_workspace(nq, base.max_ctx, 0, 0), dtype=torch.uint8, device=dev)
+          for _ in f]
+    k_per_graph = 4 * n_rep if n_rep <= 16 else n_rep
+
     def k1_call(i):
         r = i % n_rep
-        B.csa2_index_full(f[r].q, f[r].w, f[r].keys, pos_dev, pos + 1, ws=wss[r], status=status, stream=stream)
+        B.csa2_index_full(f[r].q, f[r].w, f[r].keys, replicas[r].pos_dev, base.max_ctx,
+                          seq_of_query=replicas[r].seq_dev, ws=ws[r], status=status, stream=stream)
     with torch.cuda.stream(stream):
         for i in range(n_rep):
             k1_call(i)
@@ -485,75 +546,75 @@ def run_gpu(args, rank, world, local):
     with torch.cuda.graph(kg, stream=stream):
         for i in range(k_per_graph):
             k1_call(i)
-    k_reps = max(3, args.steps // k_per_graph)
+    k_reps = max(3, 200 // k_per_graph)
     with torch.cuda.stream(stream):
         kg.replay()
-        ka, kb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ka.record(stream)
-        for _ in range(k_reps):
-            kg.replay()
-        kb.record(stream)
-    torch.cuda.synchronize()
-    k_ms = ka.elapsed_time(kb) / (k_reps * k_per_graph)
-    k_ms = max_over_ranks(k_ms, world, dev)
+    k_ms = time_replays([kg], k_reps, stream, world, dev) / k_per_graph
+    B.check_status(status)
     del kg
-    key_bytes = (pos + 1) * wl.idx_dim + wl.idx_heads * wl.idx_dim + wl.idx_heads
+    sq, qp = base.seq_of_query, base.query_pos
+    last = {}
+    for s_, p_ in zip(sq, qp):
+        last[int(s_)] = max(last.get(int(s_), -1), int(p_))
+    key_bytes = sum(p + 1 for p in last.values()) * wl.idx_dim + nq * (wl.idx_heads * wl.idx_dim + wl.idx_heads)
     pk = peaks()
     achieved = key_bytes / (k_ms / 1e3) / 1e9
 
-    # ---- end to end through the C ABI with host buffers
-    h2d = [l.q_attn for l in replicas[0]] + [t for l in replicas[0] if l.q is not None for t in (l.q, l.w)]
-    h2d_host = [t.cpu().pin_memory() for t in h2d]
-    d2h = [l.out for l in replicas[0]]
-    d2h_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in d2h]
-    h2d_bytes = sum(t.numel() * t.element_size() for t in h2d_host)
-    d2h_bytes = sum(t.numel() * t.element_size() for t in d2h_host)
-    e_steps = max(args.steps, 10)
+    # ---- end to end through the C ABI with host buffers: one pinned H2D of the
+    # step's inputs, the plan call, one D2H of its outputs
+    r0, p0 = replicas[0], plans[0]
+    in_host = r0.inbuf.cpu().pin_memory()
+    out_host = torch.empty(r0.outbuf.shape, dtype=r0.outbuf.dtype, pin_memory=True)
+
+    def e2e_step():
+        r0.inbuf.copy_(in_host, non_blocking=True)
+        p0.run(stream)
+        out_host.copy_(r0.outbuf, non_blocking=True)
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            for hsrc, ddst in zip(h2d_host, h2d):
-                ddst.copy_(hsrc, non_blocking=True)
-            plans[0].run(stream)
-            for dsrc, hdst in zip(d2h, d2h_host):
-                hdst.copy_(dsrc, non_blocking=True)
+        for _ in range(3):
+            e2e_step()
     torch.cuda.synchronize()
+    e_steps = max(args.steps, 20)
     barrier(world)
+    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for _ in range(e_steps):
-            for hsrc, ddst in zip(h2d_host, h2d):
-                ddst.copy_(hsrc, non_blocking=True)
-            plans[0].run(stream)
-            for dsrc, hdst in zip(d2h, d2h_host):
-                hdst.copy_(dsrc, non_blocking=True)
+            e2e_step()
         e1.record(stream)
     torch.cuda.synchronize()
-    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    e2e = world * e_steps / (e_ms / 1e3)
-    B.check_status(plans[0].status)
+    e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / e_steps
+    B.check_status(p0.status)
 
     gbs = alg_bytes / (ms_step / 1e3) / 1e9
-    line = {"metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "int8", "data": "synthetic", "config": config_dict(wl),
+            "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+            "config": config_dict(key, wl, n_rep, rep_bytes),
+            "timing": {"repeats": REPEATS, "steps_per_repeat": args.steps, "ms_per_step_each": tb["ms_all"],
+                       "statistic": "median"},
+            "steps100": {"replays_per_repeat": tb["replays100"], "repeats": REPEATS, "ms_per_step": tb["ms100"],
+                         "ms_per_step_each": tb["ms100_all"], "value": world * units / (tb["ms100"] / 1e3)},
             "hbm": {"algorithmic_bytes_per_step": alg_bytes, "parts": parts, "achieved_gbs": gbs,
                     "frac_of_8tbs": gbs / NOMINAL_HBM_GBS, "frac_of_measured": gbs / pk["hbm_gbs"]},
-            "roofline": {"kernel": "index_score_kernel<128,64> (full-mode index scoring of 1M keys)",
+            "roofline": {"kernel": "index_score_kernel (full-mode index scoring of every key row, scores only)",
                          "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"], "ms_per_launch": k_ms,
-                         "bytes_per_launch": key_bytes, "traffic": K1_TRAFFIC_BYTES},
-            "e2e": {"value": e2e, "unit": "steps/s", "h2d_bytes_per_step": h2d_bytes,
-                    "d2h_bytes_per_step": d2h_bytes, "path": "pinned H2D + csa2_layer_plan + D2H, no graph"},
-            "gpu_launches": kernels_per_step(wl) * args.steps,
+                         "bytes_per_launch": key_bytes, "traffic": K1_TRAFFIC_BYTES.get(key)},
+            "e2e": {"value": world * units / (e_ms / 1e3), "unit": unit, "h2d_bytes_per_step": in_host.numel(),
+                    "d2h_bytes_per_step": out_host.numel(),
+                    "path": "one pinned H2D of the packed inputs + csa2_layer_plan + one D2H of the packed outputs, "
+                            "no graph"},
+            "gpu_launches": (n_kernels or 0) * args.steps, "kernels_per_step": n_kernels,
             "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
+    if key == "verify":
+        line["verify"] = {"queries_per_block": nq, "us_per_block": ms_step * 1e3,
+                          "key_bytes_per_query": key_bytes / nq,
+                          "key_passes": "groups of 4 queries share each key tile: 2 passes per 5-query block"}
     line["device"] = device_facts(dev)
     if rank == 0 and not args.no_cpu_baseline:
-        sec, _ = OracleStep(wl, host).run(1, 0)
-        line["cpu_baseline"] = {"value": 1.0 / sec, "unit": "steps/s", "cores": cpu_cores_used(), "kind": "oracle",
-                                "sample": "one whole 8-layer decode step of the same 1M-context workload"}
-    for p in plans:
-        B.check_status(p.status)
+        line["cpu_baseline"] = cpu_baseline_decode(key)
     del graphs
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -572,47 +633,32 @@ def peak_int8_tops() -> dict:
         return {"tops": 2.0 * 1590.0, "src": "fallback bf16 x 2 (nominal int8/bf16 ratio)"}
 
 
-def prefill_replica(wl, host, dev, status):
-    """Device state of one prefill chunk: keys, FP4 cache, the queries."""
-    from kv_cache_decode_csa2_b200 import csa2 as B
-    n, q, w, qa = host
-    codes = torch.empty((n, wl.attn_dim // 2), dtype=torch.uint8, device=dev)
-    scales = torch.empty((n, wl.attn_dim // 32), dtype=torch.uint8, device=dev)
-    step = 1 << 17
-    for a in range(0, n, step):                # FP4 cache written by the library's quantiser
-        b = min(n, a + step)
-        x = torch.from_numpy(synth.kv_values(wl, 0, 0, a, b)).to(dev)
-        B.csa2_fp4_quantize(x, codes[a:b], scales[a:b], status=status)
-    keys = torch.from_numpy(synth.index_keys(wl, 0, 0)).to(dev)
-    return {"keys": B.Rows(keys), "codes": B.Rows(codes), "scales": B.Rows(scales),
-            "q": torch.from_numpy(q).to(dev), "w": torch.from_numpy(w).to(dev),
-            "qa": torch.from_numpy(qa).to(dev).to(torch.bfloat16)}
+PREFILL_SAMPLE = "the chunk's last query (its whole 262,144-row prefix), through the oracle"
 
 
-PREFILL_SAMPLE = "the chunk's last query (its whole 262,144-row prefix), through the oracle one query at a time"
-
-
-def prefill_host(wl):
-    n = int(wl.lengths()[0])
-    _, qp = wl.query_positions()
-    qs = [synth.index_query(wl, 0, i) for i in range(len(qp))]
-    return (n, np.stack([x[0] for x in qs]), np.stack([x[1] for x in qs]),
-            np.stack([synth.attn_query(wl, 0, i) for i in range(len(qp))]))
-
-
-def oracle_prefill_query_seconds(wl, host, qp) -> float:
+def oracle_prefill_query_seconds(wl, host, qp, threads: int) -> float:
     """Seconds the oracle takes for one query of the chunk (the last, whose
-    prefix is the whole context): its scores, its top-k and its attention.
-    The FP4 rows of its attention set are stored, untimed, in between."""
+    prefix is the whole context): its scores (split over `threads` host
+    threads by row slices), its top-k and its attention.  The FP4 rows of
+    its attention set are stored, untimed, in between."""
     import oracle as O
+    from concurrent.futures import ThreadPoolExecutor
+
     from threadpoolctl import threadpool_limits
     keys = synth.index_keys(wl, 0, 0)
     i = len(qp) - 1
     pos = int(qp[i])
-    with threadpool_limits(1):
+    n = pos + 1
+    with threadpool_limits(threads):
         t0 = time.perf_counter()
-        s_ = O.index_scores(host[1][i], host[2][i], keys[:pos + 1])
-        sel_ = O.top_k_positions(s_, np.arange(pos + 1), wl.topk)
+        if threads > 1:
+            cuts = [n * j // threads for j in range(threads + 1)]
+            with ThreadPoolExecutor(threads) as ex:
+                s_ = np.concatenate(list(ex.map(
+                    lambda j: O.index_scores(host[1][i], host[2][i], keys[cuts[j]:cuts[j + 1]]), range(threads))))
+        else:
+            s_ = O.index_scores(host[1][i], host[2][i], keys[:n])
+        sel_ = O.top_k_positions(s_, np.arange(n), wl.topk)
         S = O.attention_set(sel_, pos, wl.window)
         t1 = time.perf_counter()
         x = np.concatenate([synth.kv_values(wl, 0, 0, int(r_), int(r_) + 1) for r_ in S])
@@ -623,37 +669,38 @@ def oracle_prefill_query_seconds(wl, host, qp) -> float:
     return (t1 - t0) + (t3 - t2)
 
 
-def run_reference_prefill(args, rank, world):
-    if rank != 0:
-        return
+def run_reference_prefill(args):
+    from kv_cache_decode_csa2_b200 import workloads as W
     wl = WL_PREFILL
-    host = prefill_host(wl)
+    host = W.prefill_host(wl)
     _, qp = wl.query_positions()
-    ts = [oracle_prefill_query_seconds(wl, host, qp) for _ in range(max(1, min(args.steps, 3)))]
-    v = 1.0 / (sum(ts) / len(ts))
+    cores = host_cores()
+    ts = [oracle_prefill_query_seconds(wl, host, qp, cores) for _ in range(max(1, min(args.steps, 5)))]
+    v = 1.0 / statistics.median(ts)
     line = {"impl": "reference", "metric": METRIC_PREFILL, "value": v, "unit": "queries/s", "n_gpus": args.gpus,
             "steps": len(ts), "warmup": 0, "ms_per_step": 1e3 / v, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "int64,f64", "data": "synthetic",
             "config": {"workload": wl.name},
-            "cpu_baseline": {"value": v, "unit": "queries/s", "cores": cpu_cores_used(), "kind": "oracle",
-                             "sample": PREFILL_SAMPLE},
+            "cpu_baseline": {"value": v, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                             "sample": PREFILL_SAMPLE, "cpu_model": cpu_model()},
             "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 def run_prefill(args, rank, world, local):
     from kv_cache_decode_csa2_b200 import csa2 as B
+    from kv_cache_decode_csa2_b200 import workloads as W
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     wl = WL_PREFILL
     t_setup = time.time()
     sq, qp = wl.query_positions()
     nq = len(qp)
-    host = prefill_host(wl)
+    host = W.prefill_host(wl)
     n = host[0]
     status = B.new_status(dev)
-    n_rep = max(1, args.replicas)
-    reps = [prefill_replica(wl, host, dev, status) for _ in range(n_rep)]
+    n_rep = args.replicas or 4
+    reps = [W.prefill_replica(wl, host, dev, status) for _ in range(n_rep)]
     pos_dev = torch.from_numpy(qp.astype(np.int32)).to(dev)
     seq_dev = torch.from_numpy(sq.astype(np.int32)).to(dev)
     sel = torch.empty((nq, wl.topk), dtype=torch.int32, device=dev)
@@ -679,6 +726,7 @@ def run_prefill(args, rank, world, local):
             attend(r)
     torch.cuda.synchronize()
     B.check_status(status)
+    n_kernels = kernels_in(lambda: (index(reps[0]), attend(reps[0])), stream)
     graphs, igraphs = [], []
     for r in reps:
         g = torch.cuda.CUDAGraph()
@@ -692,26 +740,16 @@ def run_prefill(args, rank, world, local):
         igraphs.append(gi)
     torch.cuda.synchronize()
     setup_s = time.time() - t_setup
-
-    def timed(gs, steps):
-        with torch.cuda.stream(stream):
-            for i in range(args.warmup):
-                gs[i % n_rep].replay()
-        torch.cuda.synchronize()
-        barrier(world)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            a.record(stream)
-            for i in range(steps):
-                gs[i % n_rep].replay()
-            b.record(stream)
-        torch.cuda.synchronize()
-        return max_over_ranks(a.elapsed_time(b), world, dev) / steps
-
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % n_rep].replay()
+    torch.cuda.synchronize()
     with ClockSampler(gpu_id(dev)) as clk:
-        time.sleep(0.3)
-        ms = timed(graphs, args.steps)
-    ms_index = timed(igraphs, max(3, args.steps))
+        load_for(graphs, 0.4, stream)
+        per = [time_replays(graphs, args.steps, stream, world, dev) for _ in range(REPEATS)]
+    ms = statistics.median(per)
+    ms_index = statistics.median([time_replays(igraphs, max(3, args.steps), stream, world, dev)
+                                  for _ in range(REPEATS)])
     B.check_status(status)
     ops = sum((int(p) + 1) * wl.idx_heads * wl.idx_dim * 2 for p in qp)
     tops = ops / (ms_index / 1e3) / 1e12
@@ -747,7 +785,9 @@ def run_prefill(args, rank, world, local):
                        "kv": f"FP4 E2M1 d{wl.attn_dim}, E4M3 per 32", "q_heads": wl.attn_heads,
                        "l2": f"inputs rotate over {n_rep} device replicas (~180 MB each)",
                        "parallelism": "one chunk per rank"},
-            "roofline": {"kernel": "index stage: index_score_kernel<128,64,4> + per-query top-512",
+            "timing": {"repeats": REPEATS, "steps_per_repeat": args.steps, "ms_per_step_each": per,
+                       "statistic": "median"},
+            "roofline": {"kernel": "index stage: grouped index_score_kernel + per-query top-512",
                          "bound": "tensor", "achieved": tops, "peak": pk["tops"], "unit": "TOP/s (int8)",
                          "frac": tops / pk["tops"], "peak_src": pk["src"], "ms_per_launch": ms_index,
                          "ops_per_launch": ops, "traffic": None},
@@ -755,12 +795,13 @@ def run_prefill(args, rank, world, local):
                     "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in h2d_host),
                     "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in d2h_host),
                     "path": "pinned H2D + csa2_index_full + csa2_sparse_attn_fp4 + D2H, no graph"},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": (n_kernels or 0) * args.steps, "kernels_per_step": n_kernels,
             "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
     if rank == 0 and not args.no_cpu_baseline:
-        sec = oracle_prefill_query_seconds(wl, host, qp)
-        line["cpu_baseline"] = {"value": 1.0 / sec, "unit": "queries/s", "cores": cpu_cores_used(), "kind": "oracle",
-                                "sample": PREFILL_SAMPLE}
+        cores = host_cores()
+        sec = oracle_prefill_query_seconds(wl, host, qp, cores)
+        line["cpu_baseline"] = {"value": 1.0 / sec, "unit": "queries/s", "cores": cores, "kind": "oracle",
+                                "sample": PREFILL_SAMPLE, "cpu_model": cpu_model()}
     del graphs, igraphs
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -773,31 +814,37 @@ def quant_bytes_per_row(D: int) -> int:
     return 2 * D + D // 2 + D // 32
 
 
-def oracle_quant_rows_per_s(wl, rows: int) -> tuple[float, str]:
+def oracle_quant_rows_per_s(wl, rows: int, threads: int) -> tuple[float, str]:
     """The oracle's FP4 quantiser on the first ``rows`` rows of layer 0 (bf16
-    values), timed on one host core."""
+    values), split into `threads` row slices on host threads."""
     import oracle as O
+    from concurrent.futures import ThreadPoolExecutor
+
     from threadpoolctl import threadpool_limits
     x = synth.round_to_bf16(synth.kv_values(wl, 0, 0, 0, rows))
+    cuts = [rows * j // threads for j in range(threads + 1)]
     with threadpool_limits(1):
         t0 = time.perf_counter()
-        O.fp4_quantize(x)
+        if threads > 1:
+            with ThreadPoolExecutor(threads) as ex:
+                list(ex.map(lambda j: O.fp4_quantize(x[cuts[j]:cuts[j + 1]]), range(threads)))
+        else:
+            O.fp4_quantize(x)
         t = time.perf_counter() - t0
-    return rows / t, f"{rows} bf16 rows of d{wl.attn_dim} of the same cache, one call"
+    return rows / t, f"{rows} bf16 rows of d{wl.attn_dim} of the same cache, split over {threads} host threads"
 
 
-def run_reference_quantize(args, rank, world):
-    if rank != 0:
-        return
+def run_reference_quantize(args):
     wl = WL
-    vs = [oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS)[0] for _ in range(max(1, min(args.steps, 3)))]
-    v = sum(vs) / len(vs)
+    cores = host_cores()
+    vs = [oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS, cores)[0] for _ in range(max(1, min(args.steps, 5)))]
+    v = statistics.median(vs)
     line = {"impl": "reference", "metric": METRIC_QUANT, "value": v, "unit": "rows/s", "n_gpus": args.gpus,
             "steps": len(vs), "warmup": 0, "ms_per_step": 1e3 * (1 << 20) / v, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": "fp4_cache_write_1m_rows_d512"},
-            "cpu_baseline": {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle",
-                             "sample": f"{QUANT_SAMPLE_ROWS} rows per step"},
+            "cpu_baseline": {"value": v, "unit": "rows/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{QUANT_SAMPLE_ROWS} rows per step", "cpu_model": cpu_model()},
             "e2e": {"value": v, "unit": "rows/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -834,19 +881,10 @@ def run_quantize(args, rank, world, local):
         for _ in range(args.warmup):
             g.replay()
     torch.cuda.synchronize()
-    barrier(world)
-    torch.cuda.synchronize()
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id(dev)) as clk:
-        time.sleep(0.3)
-        with torch.cuda.stream(stream):
-            ev0.record(stream)
-            for _ in range(args.steps):
-                g.replay()
-            ev1.record(stream)
-        torch.cuda.synchronize()
-    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / args.steps
-    barrier(world)
+        load_for([g], 0.4, stream)
+        per = [time_replays([g], args.steps, stream, world, dev) for _ in range(REPEATS)]
+    ms = statistics.median(per)
     B.check_status(status)
     per_row = quant_bytes_per_row(D)
     achieved = n * per_row / (ms / 1e3) / 1e9
@@ -875,6 +913,8 @@ def run_quantize(args, rank, world, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16->fp4", "data": "synthetic",
             "config": {"workload": "fp4_cache_write_1m_rows_d512", "rows": n, "d": D, "input": "bf16",
                        "l2": "1 GiB of input per step, far beyond L2", "parallelism": "one cache per rank"},
+            "timing": {"repeats": REPEATS, "steps_per_repeat": args.steps, "ms_per_step_each": per,
+                       "statistic": "median"},
             "roofline": {"kernel": "fp4_quantize_kernel<bf16>", "bound": "hbm", "achieved": achieved,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                          "peak_src": pk["src"], "ms_per_launch": ms, "bytes_per_launch": n * per_row,
@@ -883,42 +923,44 @@ def run_quantize(args, rank, world, local):
                     "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                     "d2h_bytes_per_step": ch.numel() + sh.numel(),
                     "path": "pinned H2D + csa2_fp4_quantize + D2H, no graph"},
-            "gpu_launches": args.steps, "clocks": clk.summary(), "setup_s": round(setup_s, 1)}
+            "gpu_launches": args.steps, "kernels_per_step": 1, "clocks": clk.summary(),
+            "setup_s": round(setup_s, 1)}
     if rank == 0 and not args.no_cpu_baseline:
-        v, sample = oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS)
-        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": 1, "kind": "oracle", "sample": sample}
+        cores = host_cores()
+        v, sample = oracle_quant_rows_per_s(wl, QUANT_SAMPLE_ROWS, cores)
+        line["cpu_baseline"] = {"value": v, "unit": "rows/s", "cores": cores, "kind": "oracle", "sample": sample,
+                                "cpu_model": cpu_model()}
     del g
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
+WORKLOAD_NAMES = list(DECODE_WORKLOADS) + ["prefill", "quantize"]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
-    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "quantize"],
-                    help="decode: the 1M-context 8-layer step (default); prefill: the 2048-query chunk; "
-                         "quantize: the FP4 cache write of 1M bf16 rows")
-    ap.add_argument("--replicas", type=int, default=N_REPLICAS,
-                    help="device copies of the state rotated between steps (4 keep each step's reads out of L2)")
+    ap.add_argument("--workload", default="decode", choices=WORKLOAD_NAMES)
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="device copies of the state rotated between steps (default: enough to exceed 2x L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_init(args.gpus)
     try:
-        if args.workload == "quantize":
-            (run_reference_quantize if args.impl == "reference" else run_quantize)(args, rank, world, *(
-                () if args.impl == "reference" else (local,)))
-        elif args.workload == "prefill":
-            (run_reference_prefill if args.impl == "reference" else run_prefill)(args, rank, world, *(
-                () if args.impl == "reference" else (local,)))
-        elif args.impl == "reference":
+        if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload == "prefill":
+            run_prefill(args, rank, world, local)
+        elif args.workload == "quantize":
+            run_quantize(args, rank, world, local)
         else:
-            run_gpu(args, rank, world, local)
+            run_decode(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

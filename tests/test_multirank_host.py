@@ -75,14 +75,13 @@ def test_single_rank_needs_no_process_group():
     bench.barrier(1)              # a no-op with one rank
 
 
-@pytest.mark.parametrize("workload", ["decode", "prefill", "quantize"])
+@pytest.mark.parametrize("workload", ["decode", "tiny", "single", "ragged", "verify", "prefill", "quantize"])
 def test_reference_arm_runs_on_rank_zero_only(workload, capsys):
     bench = _bench()
 
     class Args:
         gpus, steps, warmup, impl = 2, 1, 3, "reference"
 
-    fn = {"decode": bench.run_reference, "prefill": bench.run_reference_prefill,
-          "quantize": bench.run_reference_quantize}[workload]
-    fn(Args(), 1, 2)               # rank 1 of 2: no oracle work, no output
+    Args.workload = workload
+    bench.run_reference(Args(), 1, 2)   # rank 1 of 2: no oracle work, no output
     assert capsys.readouterr().out == ""

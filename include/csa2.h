@@ -175,7 +175,10 @@ size_t csa2_topk_pool_workspace(int32_t nq, int32_t n_max, int32_t k);
  * allows 8 queries of up to 10^6 candidates each, or 7 of up to 2^24.
  * The call allocates and frees nothing.  Its first call on a device looks up
  * the array's address there (cudaGetSymbolAddress), so make that first call
- * before any stream capture on that device.
+ * before any stream capture on that device.  The address is kept per device
+ * together with the context it was found in; after a device reset (a new
+ * context, the module loaded again) the next call looks it up again, and that
+ * call too must come before any stream capture.
  * Every call uses the same array and clears the parts that must start at
  * zero.  Calls that overlap on the GPU (other streams, other threads) race on
  * it, so serialise them.
@@ -223,7 +226,8 @@ size_t csa2_reindex_workspace(int32_t nq, int32_t P, int32_t K);
  *   out      bf16 [nq][Hq][D];  lse float [nq][Hq] or NULL (natural log of
  *            the softmax denominator, including the scale)
  * Supported: D in {128, 512}; Hq in {8, 16, ..., 128} (a multiple of 8);
- * 0 <= K <= 65536; 1 <= window <= 1024.
+ * 0 <= K <= 65536; 0 <= window <= 1024 (0: S is the selection alone, as for a
+ * context shard that holds none of the query's window rows).
  */
 int32_t csa2_sparse_attn_fp4(const uint16_t* q, const csa2_rows* codes, const csa2_rows* scales,
                              const int32_t* seq_of_query, const int32_t* query_pos,
@@ -232,6 +236,26 @@ int32_t csa2_sparse_attn_fp4(const uint16_t* q, const csa2_rows* codes, const cs
                              float softmax_scale, uint16_t* out, float* lse,
                              void* ws, size_t ws_bytes, int32_t* status, void* stream);
 size_t csa2_sparse_attn_workspace(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
+
+/* csa2_attn_combine: attention over the union of R disjoint row sets, from
+ * the R partial results over each set.  Softmax over the union is each part's
+ * softmax rescaled by its share of the total mass, so with lse_r the natural
+ * log of part r's softmax denominator (the `lse` output of
+ * csa2_sparse_attn_fp4):
+ *     LSE = log sum_r exp(lse_r),   out = sum_r exp(lse_r - LSE) o_r.
+ * This is the last step of a context-sharded decode: each part (a GPU that
+ * owns a slice of the cache) attends to the rows of S it holds; the pages
+ * scale context by selection ("DeepSeek V4.1-Flash: 552B runs like 16B",
+ * Act 2), and the selected rows then live on whichever slice holds them.
+ *   o_parts    bf16 [R][nq][Hq][D] (16-byte aligned)
+ *   lse_parts  float [R][nq][Hq]; -inf: that part holds no row of the query
+ *   out        bf16 [nq][Hq][D] (16-byte aligned); lse_out float [nq][Hq]
+ *              or NULL (-inf when no part holds a row)
+ * Accumulation is fp32.  Supported: 1 <= R <= 4096, 8 <= D <= 1024 with D a
+ * multiple of 8.  Nothing is allocated; no workspace.
+ */
+int32_t csa2_attn_combine(const uint16_t* o_parts, const float* lse_parts, int32_t R, int32_t nq, int32_t Hq,
+                          int32_t D, uint16_t* out, float* lse_out, int32_t* status, void* stream);
 
 /* csa2_sparse_attn_fp4_local: csa2_sparse_attn_fp4 for a layer that keeps its
  * own cache of the most recent tokens beside the FP4 main cache (V4 kept a

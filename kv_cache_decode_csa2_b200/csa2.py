@@ -76,6 +76,7 @@ _SIGS = {
     "csa2_layer_plan": (_I32, [_P, _I32, ctypes.POINTER(csa2_layer), ctypes.POINTER(csa2_plan_shape), _P,
                                _SZ, _P, _P]),
     "csa2_layer_plan_workspace": (_SZ, [_P, _I32, ctypes.POINTER(csa2_plan_shape)]),
+    "csa2_attn_combine": (_I32, [_P, _P, _I32, _I32, _I32, _I32, _P, _P, _P, _P]),
     "csa2_fp4_quantize": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
     "csa2_fp4_quantize_bf16": (_I32, [_P, _I64, _I32, _I64, _P, _P, _I64, _P, _I64, _I64, _P, _P]),
     "csa2_status_string": (ctypes.c_char_p, [_I32]),
@@ -278,6 +279,22 @@ def csa2_fp4_quantize(x, codes, scales, *, dst_rows=None, status=None, stream=No
     code = fn(_ptr(x), n, D, x.stride(0), _ptr(dst_rows), _ptr(codes), codes.stride(0), _ptr(scales),
               scales.stride(0), codes.shape[0], _ptr(status), _stream(stream))
     _check(code, name)
+    return status
+
+
+def csa2_attn_combine(o_parts, lse_parts, out, *, lse_out=None, status=None, stream=None):
+    """Attention over the union of R disjoint row sets from the R partial
+    results: o_parts bf16 [R][nq][Hq][D], lse_parts float32 [R][nq][Hq]."""
+    L = lib()
+    _dev(o_parts, torch.bfloat16, "o_parts")
+    _dev(lse_parts, torch.float32, "lse_parts")
+    _dev(out, torch.bfloat16, "out")
+    R, nq, Hq, D = o_parts.shape
+    if tuple(lse_parts.shape) != (R, nq, Hq) or tuple(out.shape) != (nq, Hq, D):
+        raise ValueError("csa2_attn_combine: shapes do not match")
+    status = new_status(o_parts.device) if status is None else status
+    _check(L.csa2_attn_combine(_ptr(o_parts), _ptr(lse_parts), R, nq, Hq, D, _ptr(out), _ptr(lse_out),
+                               _ptr(status), _stream(stream)), "csa2_attn_combine")
     return status
 
 

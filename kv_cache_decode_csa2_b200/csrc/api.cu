@@ -5,28 +5,10 @@
 #include <string.h>
 
 #include "csa2_device.cuh"
+#include "fused_select.cuh"
 #include "internal.h"
 
-#ifdef CSA2_TRACE
-#include <nvtx3/nvToolsExt.h>
-#endif
-
 using namespace csa2;
-
-// In the traced build every entry point opens a named NVTX range, so that a
-// profiler can attribute each kernel launch to the C call that made it (a
-// plan call nests the calls it makes).  The normal build has none.
-#ifdef CSA2_TRACE
-namespace {
-struct ApiRange {
-  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
-  ~ApiRange() { nvtxRangePop(); }
-};
-}  // namespace
-#define CSA2_API_RANGE(name) ApiRange api_range_(name)
-#else
-#define CSA2_API_RANGE(name) ((void)0)
-#endif
 
 namespace {
 
@@ -47,13 +29,27 @@ bool rows_ok(const csa2_rows* v, int64_t min_row_bytes, int64_t row_align) {
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
 
 size_t index_full_ws(int32_t nq, int32_t max_ctx, int32_t P, int32_t K, void* base, int32_t** scores,
-                     TopkScratch* ts) {
+                     TopkScratch* ts, FusedSel* fs) {
   Carver c(base);
   int32_t* sc = c.take<int32_t>((size_t)nq * (size_t)max_ctx);
   TopkScratch t{};
   if (P > 0 || K > 0) t = carve_topk(c, nq, max_ctx);
+  FusedSel f{};
+  if (nq == 1 && (P > 0 || K > 0)) {   // one query: the select may run inside the index launch
+    f.hrows = c.take<uint32_t>((size_t)kFsMaxG * kBuckets);
+    f.red = c.take<uint32_t>(kBuckets);
+    f.stot = c.take<uint32_t>(kFsMaxG);
+    f.cnts = c.take<uint32_t>((size_t)kFsMaxG * 8);
+    f.tkeys = c.take<uint64_t>((size_t)kFsMaxG * 2 * kFsOwnCap);
+    // the counts that must start at zero live in the region zeroed for the
+    // top-k anyway: the digit counts in the (then unused) histogram, the
+    // barrier in the select header
+    f.radix = t.hist;
+    f.bar = t.sel_hdr;
+  }
   if (scores) *scores = sc;
   if (ts) *ts = t;
+  if (fs) *fs = f;
   return c.used + 256;
 }
 
@@ -83,8 +79,16 @@ int32_t run_reindex(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* s
   TopkScratch ts;
   ReindexSelScratch rs;
   reindex_ws(nq, P, n_jobs, ws, &sc_ws, &ts, &rs);
+  // The co-resident fused launch when every pool's CTAs fit on the device at
+  // once; else one cluster per (layer, query) (no grid barrier, any number of
+  // pools); else scores and a select per layer.  The cluster form is second:
+  // it gathers each pool's rows with 16 SMs instead of 64 and exchanges
+  // through distributed shared memory, which measured slower for one query.
   cudaError_t e = launch_reindex_select(jobs, n_jobs, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, K, rs,
                                         status, st);
+  if (e != cudaErrorNotSupported) return cuda_status(e);
+  (void)cudaGetLastError();
+  e = launch_reindex_cluster(jobs, n_jobs, seq_of_query, pool_idx, pool_cnt, nq, H, D, P, K, status, st);
   if (e != cudaErrorNotSupported) return cuda_status(e);
   (void)cudaGetLastError();
   for (int j = 0; j < n_jobs; ++j) {
@@ -139,7 +143,8 @@ int32_t csa2_trace_attach(void* table) {
   if (table && !aligned(table, 8)) return CSA2_ERR_INVALID_ARG;
   uint64_t* t = static_cast<uint64_t*>(table);
   cudaError_t (*const attach[])(uint64_t*) = {trace_attach_index, trace_attach_select, trace_attach_reindex,
-                                               trace_attach_attn,  trace_attach_rows,   trace_attach_zero};
+                                               trace_attach_attn,  trace_attach_rows,   trace_attach_zero,
+                                               trace_attach_rcluster};
   for (auto f : attach)
     if (f(t) != cudaSuccess) return CSA2_ERR_CUDA;
   return CSA2_OK;
@@ -151,7 +156,7 @@ int32_t csa2_trace_attach(void* table) {
 
 size_t csa2_index_full_workspace(int32_t nq, int32_t max_ctx, int32_t P, int32_t K) {
   if (nq < 1 || max_ctx < 1) return 0;
-  return index_full_ws(nq, max_ctx, P, K, nullptr, nullptr, nullptr);
+  return index_full_ws(nq, max_ctx, P, K, nullptr, nullptr, nullptr, nullptr);
 }
 
 int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
@@ -174,13 +179,32 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* sc_ws;
   TopkScratch ts;
-  index_full_ws(nq, max_ctx, P, K, ws, &sc_ws, &ts);
+  FusedSel fs;
+  index_full_ws(nq, max_ctx, P, K, ws, &sc_ws, &ts, &fs);
   int32_t* sc = scores ? scores : sc_ws;
   const int64_t ld = scores ? ld_scores : max_ctx;
   const bool topk = P > 0 || K > 0;
   if (topk && !launch_opts().prezeroed) {
     cudaError_t e = cudaMemsetAsync(ts.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
+  }
+  if (topk && nq == 1) {   // one query: pool and selection inside the index launch when it fits
+    fs.on = 1;
+    fs.n_k = 0;
+    if (P > 0) {
+      fs.k[fs.n_k] = P;
+      fs.out_idx[fs.n_k] = pool_idx;
+      fs.out_cnt[fs.n_k++] = pool_cnt;
+    }
+    if (K > 0) {
+      fs.k[fs.n_k] = K;
+      fs.out_idx[fs.n_k] = sel_idx;
+      fs.out_cnt[fs.n_k++] = sel_cnt;
+    }
+    cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,
+                                       nullptr, status, st, nullptr, &fs);
+    if (e != cudaErrorNotSupported) return cuda_status(e);
+    (void)cudaGetLastError();
   }
   bool hist_built = false;
   cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,
@@ -249,7 +273,7 @@ int32_t csa2_reindex(const int8_t* q, const int8_t* w, const csa2_rows* keys,
 }
 
 size_t csa2_sparse_attn_workspace(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window) {
-  if (nq < 1 || Hq < 1 || D < 1 || K < 0 || window < 1) return 0;
+  if (nq < 1 || Hq < 1 || D < 1 || K < 0 || window < 0) return 0;
   return attn_scratch_bytes(nq, Hq, D, K, window);
 }
 
@@ -257,7 +281,7 @@ static int32_t check_attn(const uint16_t* q, const csa2_rows* codes, const csa2_
                           const int32_t* query_pos, int32_t nq, int32_t Hq, int32_t D, int32_t K,
                           int32_t window, const uint16_t* out) {
   if (!q || !query_pos || !out || !aligned(q, 16) || !aligned(out, 16)) return CSA2_ERR_INVALID_ARG;
-  if (nq < 1 || nq > 65535 || K < 0 || K > 65536 || window < 1 || window > 1024) return CSA2_ERR_INVALID_ARG;
+  if (nq < 1 || nq > 65535 || K < 0 || K > 65536 || window < 0 || window > 1024) return CSA2_ERR_INVALID_ARG;
   if (D != 128 && D != 512) return CSA2_ERR_UNSUPPORTED;
   if (Hq < 8 || Hq > 128 || Hq % 8) return CSA2_ERR_UNSUPPORTED;
   if (!rows_ok(codes, D / 2, 16) || !rows_ok(scales, D / 32, 1)) return CSA2_ERR_INVALID_ARG;
@@ -430,7 +454,7 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
     size_t zb[3];
     int nz = 0;
     TopkScratch ts;
-    index_full_ws(s->nq, s->max_ctx, s->P, s->K, p.index_base, nullptr, &ts);
+    index_full_ws(s->nq, s->max_ctx, s->P, s->K, p.index_base, nullptr, &ts, nullptr);
     zp[nz] = ts.hist;
     zb[nz++] = topk_zero_bytes(s->nq);
     if (n_reindex > 0) {
@@ -489,6 +513,18 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
   const float scale = s->softmax_scale > 0.f ? s->softmax_scale : 1.0f / sqrtf((float)s->D);
   return cuda_status(launch_sparse_attn_jobs(jobs, L, s->seq_of_query, s->query_pos, s->nq, s->Hq, s->D, s->K,
                                              s->window, scale, p.attn_base, status, st));
+}
+
+// ------------------------------------------------------------------ combine of partial attention
+int32_t csa2_attn_combine(const uint16_t* o_parts, const float* lse_parts, int32_t R, int32_t nq, int32_t Hq,
+                          int32_t D, uint16_t* out, float* lse_out, int32_t* status, void* stream) {
+  CSA2_API_RANGE("csa2_attn_combine");
+  if (!o_parts || !lse_parts || !out || !status || !aligned(o_parts, 16) || !aligned(out, 16))
+    return CSA2_ERR_INVALID_ARG;
+  if (R < 1 || R > 4096 || nq < 1 || Hq < 1 || (int64_t)nq * Hq > (1 << 26)) return CSA2_ERR_INVALID_ARG;
+  if (D < 8 || D > 1024 || D % 8) return CSA2_ERR_UNSUPPORTED;
+  return cuda_status(launch_attn_combine(o_parts, lse_parts, R, nq, Hq, D, out, lse_out,
+                                         static_cast<cudaStream_t>(stream)));
 }
 
 // ------------------------------------------------------------------ FP4 cache write

@@ -43,7 +43,8 @@ __device__ __forceinline__ uint64_t global_ns() {
 constexpr int kTraceKernels = 8;
 constexpr int kTraceCtas = 1024;
 constexpr int kTracePhases = 16;
-enum TraceKernel : int { kTrIndex = 0, kTrSelect = 1, kTrReindex = 2, kTrAttn = 3, kTrRowSel = 4, kTrZero = 5 };
+enum TraceKernel : int { kTrIndex = 0, kTrSelect = 1, kTrReindex = 2, kTrAttn = 3, kTrRowSel = 4, kTrZero = 5,
+                          kTrRCluster = 6 };
 #ifdef CSA2_TRACE
 __device__ __forceinline__ void trace_mark(uint64_t* table, int kernel, int phase, long long t0) {
   const uint32_t cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);

@@ -21,6 +21,7 @@
 // Work is the flat list of (query, 128-row tile) items over all queries,
 // split evenly between CTAs, so ragged batches stay balanced.
 #include "csa2_device.cuh"
+#include "fused_select.cuh"
 #include "internal.h"
 
 namespace csa2 {
@@ -40,6 +41,7 @@ struct IndexArgs {
   int64_t ld;
   uint32_t* hist;
   int32_t* status;
+  FusedSel fs;   // fs.on: one query's pool and selection in the same launch
 };
 
 constexpr int kMaxQueries = 4096;   // per launch (the work list prefix lives in shared memory)
@@ -103,7 +105,9 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int lane = tid & 31;
   // trace points: 1 prologue done, 2 first TMA issued, 3 first stage landed,
   // 4 first epilogue tile done, 5 last epilogue tile done, 6 histogram
-  // flushed, 7 producer done, 8 MMA issuer done, 9 exit
+  // flushed, 7 producer done, 8 MMA issuer done, 9 stream done, 10 pool and
+  // selection written, and inside the fused select: 11 rows stored, 12 slices
+  // summed, 13 thresholds, 14 counts published, 15 ties resolved
   CSA2_TRACE_BEGIN(kTrIndex, tid == 0);
 
   // ---- prologue: warp 0 builds the work list (groups of queries and the
@@ -120,7 +124,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       mbar_init(&tempty[i], kEpiThreads / 64);   // one arrival per warp of the group that reads it
     }
     mbar_init(bready, kEpiThreads / 32);
-    for (int k = 0; k < QG; ++k) bound_acc[k] = 0ull;
+    for (int k = 0; k < QG; ++k) {
+      bound_acc[k] = 0ull;
+      mpos[k] = -1;   // a CTA with no segment (no valid position) keeps -1
+    }
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -483,6 +490,20 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   CSA2_MARK(kTrIndex, 9, tid == 0);
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
   if (tid == 0 && *abort_flag) record_error(a.status, CSA2_ERR_TIMEOUT);
+  if constexpr (QG == 1) {
+    if (a.fs.on) {   // one query, one CTA per SM: the pool and selection here, after the stream
+      // this CTA's positions: its tiles [lo, hi) of the query's single group, up to the query position
+      const int32_t qp = mpos[0];
+      const int64_t p_hi64 = hi * 128 < (int64_t)qp + 1 ? hi * 128 : (int64_t)qp + 1;
+      auto mark = [&](int p) {
+        (void)p;
+        CSA2_MARK(kTrIndex, p, tid == 0);
+      };
+      fused_select<64 + kEpiThreads, (NST * TILE - kFsGather * 8) / 4>(
+          a.fs, a.scores, hist_s, stages, (int32_t)(lo * 128), (int32_t)(p_hi64 > 0 ? p_hi64 : 0), a.status, mark);
+      CSA2_MARK(kTrIndex, 10, tid == 0);
+    }
+  }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -532,11 +553,22 @@ int sm_count() {
   return n;
 }
 
+// Whether one query's pool and selection can run inside its index-score
+// launch: every CTA's positions fit in its freed key ring, and the scratch
+// covers the CTA count.
+bool fused_select_fits(int32_t D, int32_t max_ctx, int grid) {
+  const int64_t tiles = (max_ctx + 127) / 128;
+  const int64_t per_cta = (tiles + grid - 1) / grid * 128;
+  const int64_t maxp = D == 128 ? (IndexCfg<128>::kStages * IndexCfg<128>::kTile - kFsGather * 8) / 4
+                                : (IndexCfg<64>::kStages * IndexCfg<64>::kTile - kFsGather * 8) / 4;
+  return grid >= 1 && grid <= kFsMaxG && per_cta <= maxp;
+}
+
 cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st, bool* hist_built) {
+                               cudaStream_t st, bool* hist_built, const FusedSel* fs) {
   if (nq > kMaxQueries) return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -559,9 +591,14 @@ cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows
   const bool grouped = N <= 64 && (nq >= kGroupMinQueries || (launch_opts().group && nq >= 2));
   if (hist_built) *hist_built = !grouped && hist;
   IndexArgs a{q, w, seq_of_query, query_pos, to_rowmap(keys), nq, H, max_ctx, scores, ld,
-              grouped ? nullptr : hist, status};
+              grouped ? nullptr : hist, status, FusedSel{}};
   const int64_t upper = (int64_t)nq * ((max_ctx + 127) / 128);
   const int grid = (int)(upper < sm_count() ? (upper > 0 ? upper : 1) : sm_count());
+  if (fs && fs->on) {
+    if (grouped || nq != 1 || !fused_select_fits(D, max_ctx, grid)) return cudaErrorNotSupported;
+    a.fs = *fs;
+    a.hist = nullptr;   // the histogram stays in each CTA's shared memory
+  }
   if (D == 128) {
     switch (N) {
       case 16: return grouped ? launch_one<128, 16, 4>(map, a, grid, st) : launch_one<128, 16, 1>(map, a, grid, st);

@@ -9,6 +9,25 @@
 
 #include "csa2.h"
 
+#ifdef CSA2_TRACE
+#include <nvtx3/nvToolsExt.h>
+#endif
+
+// In the traced build every C entry point opens a named NVTX range, so that a
+// profiler can attribute each kernel launch to the C call that made it (a
+// plan call nests the calls it makes).  The normal build has none.
+#ifdef CSA2_TRACE
+namespace csa2 {
+struct ApiRange {
+  explicit ApiRange(const char* name) { nvtxRangePushA(name); }
+  ~ApiRange() { nvtxRangePop(); }
+};
+}  // namespace csa2
+#define CSA2_API_RANGE(name) ::csa2::ApiRange api_range_(name)
+#else
+#define CSA2_API_RANGE(name) ((void)0)
+#endif
+
 namespace csa2 {
 
 // Aligned carving of the caller's workspace.
@@ -49,6 +68,18 @@ cudaError_t launch_zero(void* const* ptrs, const size_t* bytes, int n, cudaStrea
 // Launches `kernel` with the cooperative and programmatic-dependence
 // attributes asked for.  A programmatic launch the device refuses is retried
 // once without the attribute, and programmatic launches stay off from then on.
+//
+// The kernels whose CTAs meet at grid barriers (select, fused reindex,
+// attention groups) are launched WITHOUT the cooperative attribute: on B200 a
+// cooperative grid starts only after the grid before it has completed, which
+// removes the programmatic-launch overlap (2.0-2.6 us per kernel boundary
+// against 0.8 us without it).  Their co-residency rests instead on two facts:
+// each launcher checks that the grid fits on the device at once (occupancy
+// query), and each of these kernels calls pdl_trigger() only after its own
+// pdl_wait(), so the grid after it is launched only when every one of its CTAs
+// is already resident.  A grid barrier that still waits too long (another
+// process filling the device) gives up after its bounded wait and records
+// CSA2_ERR_TIMEOUT.
 cudaError_t launch_ex(const void* kernel, void** args, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                       bool cooperative, bool pdl);
 template <class... Args>
@@ -94,11 +125,16 @@ TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);
 // K1: scores of every visible position for every query (tcgen05 int8), plus
 // the bucket histogram.  hist may be NULL.  *hist_built (if given) says
 // whether the histogram was built: launches of many queries leave it out.
+// With fs (fs->on), one query's pool and selection run in the same launch
+// after the stream (fused_select.cuh); returns cudaErrorNotSupported, having
+// queued nothing, when that does not fit (see fused_select_fits).
+struct FusedSel;
 cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st, bool* hist_built = nullptr);
+                               cudaStream_t st, bool* hist_built = nullptr, const FusedSel* fs = nullptr);
+bool fused_select_fits(int32_t D, int32_t max_ctx, int grid);
 
 // Radix top-k over score rows.  ks[0..n_k) are the wanted counts (n_k <= 2,
 // ks[0] >= ks[1]); outputs go to out_idx[t]/out_cnt[t].  If hist_ready, the
@@ -178,6 +214,15 @@ cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, co
                                   int32_t D, int32_t P, int32_t K, const ReindexSelScratch& r,
                                   int32_t* status, cudaStream_t st);
 
+// K3 on thread-block clusters (reindex_cluster.cu): scores and top-K of up to
+// kMaxReindexJobs reindex layers of one pool, one cluster per (layer, query),
+// no grid barrier and no scratch.  Returns cudaErrorNotSupported, having
+// queued nothing, for pools above 16 x 1024 slots, more than 64 heads, or
+// when no cluster of the size needed fits the device.
+cudaError_t launch_reindex_cluster(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* seq_of_query,
+                                   const int32_t* pool_idx, const int32_t* pool_cnt, int32_t nq, int32_t H,
+                                   int32_t D, int32_t P, int32_t K, int32_t* status, cudaStream_t st);
+
 // K4: FP4 sparse attention (local_kv: the layer's local window cache, or nullptr).
 size_t attn_scratch_bytes(int32_t nq, int32_t Hq, int32_t D, int32_t K, int32_t window);
 cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const csa2_rows& scales,
@@ -186,6 +231,11 @@ cudaError_t launch_sparse_attn(const uint16_t* q, const csa2_rows& codes, const 
                                int32_t Hq, int32_t D, int32_t K, int32_t window, float scale,
                                uint16_t* out, float* lse, void* ws, size_t ws_bytes,
                                int32_t* status, cudaStream_t st);
+
+// Combine of R partial attention results (o_r, lse_r) over disjoint row sets
+// of the same queries into attention over their union (attn_combine.cu).
+cudaError_t launch_attn_combine(const uint16_t* o, const float* lse, int32_t R, int32_t nq, int32_t Hq, int32_t D,
+                                uint16_t* out, float* lse_out, cudaStream_t st);
 
 // K7: FP4 quantiser.
 cudaError_t launch_fp4_quantize(const void* x, bool bf16, int64_t n_rows, int32_t D, int64_t ld_x,
@@ -207,6 +257,7 @@ cudaError_t trace_attach_reindex(uint64_t* table);
 cudaError_t trace_attach_attn(uint64_t* table);
 cudaError_t trace_attach_rows(uint64_t* table);
 cudaError_t trace_attach_zero(uint64_t* table);
+cudaError_t trace_attach_rcluster(uint64_t* table);
 #endif
 
 // One-time, per-device set-up (a kernel's shared-memory limit, an occupancy

@@ -196,7 +196,9 @@ template <int D, int N, int T>
 struct RSelLayout {
   static constexpr int NT = 128 * T;
   static constexpr size_t tiles = (size_t)(T * 128 * D + N * D);
-  static constexpr size_t region = tiles > (size_t)kRTieCap * 8 ? tiles : (size_t)kRTieCap * 8;
+  static constexpr size_t ties_or_hist = (size_t)kRTieCap * 8 > (size_t)kBuckets * 4 ? (size_t)kRTieCap * 8
+                                                                                      : (size_t)kBuckets * 4;
+  static constexpr size_t region = tiles > ties_or_hist ? tiles : ties_or_hist;   // reused after scoring
   static constexpr size_t smem = 1024 + region + 128 * 4 + NT * 8 + 64;
   static constexpr uint32_t cols = T * N <= 32 ? 32 : T * N <= 64 ? 64 : T * N <= 128 ? 128 : 256;
 };
@@ -348,11 +350,26 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   }
   if (J.scores && valid) J.scores[(int64_t)q * a.P + slot] = s;
 
-  // ---- the pool's bucket histogram, then the threshold bucket
+  // ---- the pool's bucket histogram, then the threshold bucket.  The CTA
+  // counts its scores in shared memory first (the tiles are free now) and
+  // adds each populated bucket to the global histogram once: global atomics
+  // on one address serialise, so one add per (CTA, bucket) instead of one per
+  // score shortens this phase.
   uint32_t* hist = a.hist + (size_t)prob * kBuckets;
   uint32_t* hdr = a.hdr + (size_t)prob * 4;
   const int32_t bk = (int32_t)score_bucket(s);
-  if (valid) atomicAdd(&hist[bk], 1u);
+  {
+    static_assert(kBuckets * 4 <= Lay::region, "the shared histogram fits in the tile region");
+    uint32_t* hs = reinterpret_cast<uint32_t*>(smem);
+    for (int i = tid; i < kBuckets; i += NT) hs[i] = 0u;
+    __syncthreads();
+    if (valid) atomicAdd(&hs[bk], 1u);
+    __syncthreads();
+    for (int i = tid; i < kBuckets; i += NT) {
+      const uint32_t v = hs[i];
+      if (v) atomicAdd(&hist[i], v);
+    }
+  }
   uint32_t phase = 0;
   sel_grid_sync(&hdr[0], ++phase * G, a.status);
   CSA2_MARK(kTrReindex, 5, tid == 0);
@@ -485,7 +502,7 @@ cudaError_t launch_rs_t(const RSelArgs& a_in, int n_jobs, int nq, size_t zero_by
     e = cudaMemsetAsync(a.hist, 0, zero_bytes, st);   // histograms and barrier headers
     if (e != cudaSuccess) return e;
   }
-  return launch_k(reindex_select_kernel<D, N, T>, dim3(a.G, nq, n_jobs), dim3(Lay::NT), smem, st, true,
+  return launch_k(reindex_select_kernel<D, N, T>, dim3(a.G, nq, n_jobs), dim3(Lay::NT), smem, st, false,
                   launch_opts().pdl, a);
 }
 

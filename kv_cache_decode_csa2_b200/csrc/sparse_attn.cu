@@ -17,7 +17,7 @@
 // Q K^T and the unnormalised P V on bf16 tensor cores with fp32 accumulation,
 // tile by tile with an online softmax, and writes its partial (max, sum, O)
 // per head to L2.  When all CTAs of the launch fit on the device at once
-// (cooperative launch), the group meets at a bounded barrier and CTA r merges
+// (checked at launch), the group meets at a bounded barrier and CTA r merges
 // columns [r D / kCl, (r + 1) D / kCl) of every head; otherwise a merge kernel
 // does the same.  Several layers of a plan go into one launch (a job array),
 // so independent layers run side by side.
@@ -573,7 +573,7 @@ cudaError_t launch_attn_t(AttnArgs& a, cudaStream_t st) {
       e = cudaMemsetAsync(a.bar, 0, (size_t)grid.y * grid.z * sizeof(uint32_t), st);
       if (e != cudaSuccess) return e;
     }
-    return launch_k(sparse_attn_kernel<D, HG, NTHR, LOCAL>, grid, dim3(NTHR), L::total, st, true,
+    return launch_k(sparse_attn_kernel<D, HG, NTHR, LOCAL>, grid, dim3(NTHR), L::total, st, false,
                     launch_opts().pdl, a);
   }
   sparse_attn_kernel<D, HG, NTHR, LOCAL><<<grid, NTHR, L::total, st>>>(a);

@@ -9,6 +9,8 @@
 // for more than 16,384 candidates.  This entry point takes its scratch from
 // one fixed array in the library's own device memory instead.  Every GPU that
 // loads the library holds the array until the process exits.
+#include <mutex>
+
 #include "csa2_device.cuh"
 #include "internal.h"
 
@@ -20,19 +22,50 @@ constexpr size_t kNoallocScratchBytes = (size_t)CSA2_NOALLOC_SCRATCH_BYTES;
 // a device address: the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_topk_scratch[kNoallocScratchBytes];
 
-std::atomic<void*> g_scratch_addr[64];   // device address of g_topk_scratch, per device id (set-up once)
+// The array's device address per device, with the context it was looked up
+// in: a device reset (or a new primary context) reloads the module, and the
+// array may then sit elsewhere, so a changed context means a new look-up.
+struct ScratchAddr {
+  CUcontext ctx = nullptr;
+  void* addr = nullptr;
+};
+ScratchAddr g_scratch[64];
+std::mutex g_scratch_mu;
 
-// Looks up the array's address on the current device the first time the
-// entry point runs there.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current_fn() {
+  static std::atomic<CtxGetCurrentFn> cached{nullptr};
+  CtxGetCurrentFn fn = cached.load(std::memory_order_acquire);
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<CtxGetCurrentFn>(p);
+      cached.store(fn, std::memory_order_release);
+    }
+  }
+  return fn;
+}
+
+// The array's address on the current device, looked up the first time the
+// entry point runs in this device's current context.
 int32_t scratch_for_current_device(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return CSA2_ERR_CUDA;
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (!get || get(&ctx) != CUDA_SUCCESS) return CSA2_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  ScratchAddr& s = g_scratch[dev];
+  if (!ctx || s.ctx != ctx || !s.addr) {
+    void* p = nullptr;   // the look-up also makes the device's primary context current if none was
     if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess || !p) return CSA2_ERR_CUDA;
-    g_scratch_addr[dev] = p;
+    if (!ctx && (get(&ctx) != CUDA_SUCCESS || !ctx)) return CSA2_ERR_CUDA;
+    s.ctx = ctx;
+    s.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = s.addr;
   return CSA2_OK;
 }
 
@@ -42,6 +75,7 @@ extern "C" int32_t csa2_topk_pool_noalloc(const int32_t* scores, int64_t ld, con
                                           const int32_t* cand_pos, int32_t nq, int32_t n_max, int32_t k,
                                           int32_t* out_idx, int32_t* out_cnt, int32_t* status, void* stream) {
   using namespace csa2;
+  CSA2_API_RANGE("csa2_topk_pool_noalloc");
   if (!out_idx || !status || nq < 1 || n_max < 0 || n_max > (1 << 30) || k < 1 || k > 65536)
     return CSA2_ERR_INVALID_ARG;
   if (n_max > 0 && (!scores || ld < n_max)) return CSA2_ERR_INVALID_ARG;

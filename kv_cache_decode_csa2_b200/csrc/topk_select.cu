@@ -8,7 +8,7 @@
 //
 // One CTA of kSelNT threads covers kSelSpan consecutive candidates, kSelPer
 // per thread, held in registers.  A row of n candidates takes G =
-// ceil(n / kSelSpan) CTAs; for G > 1 they are co-resident (cooperative
+// ceil(n / kSelSpan) CTAs; for G > 1 they are co-resident (checked at
 // launch) and meet at two grid barriers.
 //   1. threshold bucket b* from the 13-bit bucket histogram of the row (given,
 //      or built here when G == 1): every thread owns 8 bins, one block scan
@@ -423,8 +423,8 @@ cudaError_t launch_select(const int32_t* scores, int64_t ld, const int32_t* n_va
   }
   a.status = status;
   const bool pdl = launch_opts().pdl;
-  return one ? launch_k(select_kernel<16>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, G > 1, pdl, a)
-             : launch_k(select_kernel<8>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, G > 1, pdl, a);
+  return one ? launch_k(select_kernel<16>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, false, pdl, a)
+             : launch_k(select_kernel<8>, dim3(G, nq, 1), dim3(kSelNT), kSelSmem, st, false, pdl, a);
 }
 
 }  // namespace csa2

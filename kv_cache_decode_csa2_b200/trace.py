@@ -3,8 +3,8 @@
     python -m kv_cache_decode_csa2_b200.trace [--workload decode|prefill] [--warmup W] [--save T.npy]
 
 Builds libcsa2_trace.so (the library with its phase markers compiled in, see
-csa2_trace_attach in include/csa2.h), sets up the bench's workload through it,
-replays the work in a CUDA graph as the bench does, and records one replay
+csa2_trace_attach in include/csa2.h), sets up the benchmark's workload (workloads.py) through it,
+replays the work in a CUDA graph as the benchmark does, and records one replay
 after an L2 flush.  It prints, per kernel in launch order, when its CTAs
 started and reached each marked point, relative to the start of the first
 kernel: the median and the latest CTA.  Times inside a CTA come from its SM
@@ -18,7 +18,6 @@ here.
 from __future__ import annotations
 
 import argparse
-import importlib.util
 import os
 from dataclasses import dataclass
 
@@ -33,7 +32,8 @@ POINTS = 16
 POINT_NAMES = {
     0: ("index_score", ["entry", "prologue done", "first TMA issued", "first stage landed",
                         "first epilogue tile", "last epilogue tile", "histogram flushed", "producer done",
-                        "MMA issuer done", "exit"]),
+                        "MMA issuer done", "stream done", "pool and selection written", "fs rows stored",
+                        "fs slices summed", "fs thresholds", "fs counts published", "fs ties resolved"]),
     1: ("select", ["entry", "grid before done", "threshold buckets", "classified", "first grid barrier",
                    "row ties staged", "ties ranked", "second grid barrier", "written"]),
     2: ("reindex_select", ["entry", "own inputs staged", "grid before done", "pool rows gathered", "scored",
@@ -43,6 +43,9 @@ POINT_NAMES = {
                         "softmax", "P V done", "partial written", "group barrier", "merged"]),
     4: ("row_select", ["entry", "threshold buckets", "score bounds", "classified", "ties resolved", "written"]),
     5: ("zero", ["entry", "done"]),
+    6: ("reindex_cluster", ["entry", "own inputs staged", "grid before done", "rows gathered", "scored",
+                            "histogram barrier", "slice barrier", "threshold", "count barrier", "ties resolved",
+                            "written"]),
 }
 
 
@@ -129,14 +132,6 @@ def format_report(stats: list[KernelStat], ghz: float) -> str:
 
 
 # ----------------------------------------------------------------- running a workload
-def _bench_module():
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    spec = importlib.util.spec_from_file_location("csa2_bench_workloads", os.path.join(root, "bench.py"))
-    mod = importlib.util.module_from_spec(spec)
-    spec.loader.exec_module(mod)
-    return mod
-
-
 def load_traced_library():
     """Builds and loads libcsa2_trace.so in place of libcsa2.so."""
     from . import build as _build
@@ -147,26 +142,26 @@ def load_traced_library():
     return B.lib()
 
 
-def _decode_work(bench, dev, status):
-    from . import csa2 as B
-    wl = bench.WL
-    host = bench.host_inputs(wl)
-    pos = host[0]
-    layers = bench.build_device_state(wl, host, dev, status)
-    pos_dev = torch.tensor([pos], dtype=torch.int32, device=dev)
-    plan = B.LayerPlan(list(wl.modes), layers, query_pos=pos_dev, max_ctx=pos + 1, P=wl.pool, K=wl.topk,
-                       window=wl.window)
+def _decode_work(dev, status):
+    import synth
+
+    from . import workloads as W
+    st = W.build_decode(synth.C2_1M_PLAN, dev, status)
+    plan = W.decode_plan(st)
     return plan.run, [plan.status]
 
 
-def _prefill_work(bench, dev, status, stream):
+def _prefill_work(dev, status, stream):
+    import synth
+
     from . import csa2 as B
-    wl = bench.WL_PREFILL
+    from . import workloads as W
+    wl = synth.C4_PREFILL
     sq, qp = wl.query_positions()
     nq = len(qp)
-    host = bench.prefill_host(wl)
+    host = W.prefill_host(wl)
     n = host[0]
-    r = bench.prefill_replica(wl, host, dev, status)
+    r = W.prefill_replica(wl, host, dev, status)
     pos_dev = torch.from_numpy(qp.astype(np.int32)).to(dev)
     seq_dev = torch.from_numpy(sq.astype(np.int32)).to(dev)
     sel = torch.empty((nq, wl.topk), dtype=torch.int32, device=dev)
@@ -195,15 +190,14 @@ def main(argv=None) -> int:
     from . import csa2 as B
     dev = torch.device("cuda:0")
     torch.cuda.set_device(dev)
-    bench = _bench_module()
     status = B.new_status(dev)
     stream = torch.cuda.Stream(device=dev)
     table = torch.zeros(L.csa2_trace_table_bytes() // 8, dtype=torch.int64, device=dev)
     B._check(L.csa2_trace_attach(table.data_ptr()), "csa2_trace_attach")
     if args.workload == "decode":
-        run, statuses = _decode_work(bench, dev, status)
+        run, statuses = _decode_work(dev, status)
     else:
-        run, statuses = _prefill_work(bench, dev, status, stream)
+        run, statuses = _prefill_work(dev, status, stream)
     with torch.cuda.stream(stream):
         run()                                   # ordinary call first (one-time kernel set-up)
     torch.cuda.synchronize()

@@ -158,3 +158,14 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(B, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError):
         B.lib()
+
+
+def test_noalloc_capacity_matches_its_documented_bounds():
+    """The fixed array of csa2_topk_pool_noalloc holds the scratch of 8 queries
+    of up to 10^6 candidates or 7 of up to 2^24, and not one query more."""
+    L = B.lib()
+    cap = 4 << 20
+    for nq, n in [(8, 10 ** 6), (7, 2 ** 24), (2, 4194304)]:
+        assert L.csa2_topk_pool_workspace(nq, n, 16384) <= cap, (nq, n)
+    for nq, n in [(9, 10 ** 6), (8, 2 ** 24)]:
+        assert L.csa2_topk_pool_workspace(nq, n, 16384) > cap, (nq, n)

@@ -463,3 +463,38 @@ def test_sparse_attention_long_selection():
     ref, _ = O.sparse_attention(c.host_qa[(0, 0)], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
     ok, err = G.tol_ok(_np(ly.out.float())[0], ref)
     assert ok, f"max abs err {err}"
+
+
+# ------------------------------------------------------------------ one query: pool and selection fused
+# into the index launch.  Random scores leave a few ties at the threshold
+# (gathered and ranked); zero keys make every score 0 (the ties of one CTA
+# overflow its slot and the grid's radix select decides); half-zero keys with
+# a pool larger than the positive rows split a long tie list of zeros.
+@pytest.mark.parametrize("ctx,mode,P,K", [(40000, "random", 16384, 512), (40000, "zero", 16384, 512),
+                                          (40000, "half", 30000, 512), (4096, "zero", 1024, 64),
+                                          (300000, "random", 16384, 512)])
+def test_index_full_one_query_ties(ctx, mode, P, K):
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(ctx,), pool=P, topk=K)
+    c = G.build(wl, fp4_on_gpu=True)   # only the index side is checked here
+    ly = c.layers_dev[0]
+    keys = c.host_keys[(0, 0)].copy()
+    if mode == "zero":
+        keys[:] = 0
+    elif mode == "half":
+        keys[::2] = 0
+    ly.keys.data[:ctx].copy_(torch.from_numpy(keys))
+    pool = torch.full((1, P), -7, dtype=torch.int32, device=DEV)
+    pcnt = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    sel = torch.full((1, K), -7, dtype=torch.int32, device=DEV)
+    scnt = torch.full((1,), -7, dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_index_full(ly.q, ly.w, ly.keys, c.pos_dev, c.max_ctx, P=P, pool_idx=pool,
+                                     pool_cnt=pcnt, K=K, sel_idx=sel, sel_cnt=scnt))
+    q, w = c.host_q[(0, 0)]
+    _, ref_pool, ref_sel = O.full_index(q, w, keys, int(c.query_pos[0]), P, K)
+    n = int(_np(pcnt)[0])
+    assert n == len(ref_pool) and np.array_equal(_np(pool)[0, :n], ref_pool)
+    assert (_np(pool)[0, n:] == -1).all()
+    m = int(_np(scnt)[0])
+    assert m == len(ref_sel) and np.array_equal(_np(sel)[0, :m], ref_sel)
+    if mode == "zero":
+        assert np.array_equal(ref_pool, np.arange(min(P, ctx)))   # equal scores: the lowest positions

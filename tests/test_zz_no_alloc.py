@@ -35,16 +35,20 @@ def _call_ws(L, scores, n_valid, k, out, cnt, status):
                             torch.cuda.current_stream().cuda_stream)
 
 
-@pytest.mark.parametrize("n,k,spread", [(300000, 16384, 25000), (16384, 512, 40)])
-def test_noalloc_matches_workspace_entry_point_twice(n, k, spread):
+# Sizes: co-resident select CTAs (300,000 candidates), the one-CTA path
+# (16,384), and rows too long for the co-resident select (4,194,304: the
+# multi-pass path, whose chunk counts and candidate lists take most of the
+# fixed array).
+@pytest.mark.parametrize("nq,n,k,spread", [(3, 300000, 16384, 25000), (3, 16384, 512, 40),
+                                           (2, 4194304, 16384, 10 ** 6)])
+def test_noalloc_matches_workspace_entry_point_twice(nq, n, k, spread):
     if not torch.cuda.is_available():
         pytest.skip("needs a CUDA device")
     L = B.lib()
     rng = np.random.default_rng(n)
-    nq = 3
     for call in range(2):          # two calls in a row, different data each time
         s = rng.integers(-spread, spread + 1, size=(nq, n)).astype(np.int32) + 10 ** 5 * call
-        nv = np.array([n, n // 3, n - 7], dtype=np.int32)
+        nv = np.array([n, n // 3, n - 7][:nq], dtype=np.int32)
         scores = torch.from_numpy(s).cuda()
         n_valid = torch.from_numpy(nv).cuda()
         outs = []

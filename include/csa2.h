@@ -317,7 +317,9 @@ typedef struct csa2_plan_shape {
   int32_t group_queries;           /* nonzero: consecutive queries of one sequence
                                       (a speculative-verify block) share each key tile
                                       of the index scans in groups of four, from 2
-                                      queries on; zero: only from 16 queries on */
+                                      queries on; zero: every query scans alone (a
+                                      batch of distinct sequences: one query per
+                                      segment, with the fused histogram) */
 } csa2_plan_shape;
 
 int32_t csa2_layer_plan(const int32_t* modes /* host [L] */, int32_t L,

@@ -5,7 +5,6 @@
 #include <string.h>
 
 #include "csa2_device.cuh"
-#include "fused_select.cuh"
 #include "internal.h"
 
 using namespace csa2;
@@ -29,27 +28,13 @@ bool rows_ok(const csa2_rows* v, int64_t min_row_bytes, int64_t row_align) {
 int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA2_OK : CSA2_ERR_CUDA; }
 
 size_t index_full_ws(int32_t nq, int32_t max_ctx, int32_t P, int32_t K, void* base, int32_t** scores,
-                     TopkScratch* ts, FusedSel* fs) {
+                     TopkScratch* ts) {
   Carver c(base);
   int32_t* sc = c.take<int32_t>((size_t)nq * (size_t)max_ctx);
   TopkScratch t{};
   if (P > 0 || K > 0) t = carve_topk(c, nq, max_ctx);
-  FusedSel f{};
-  if (nq == 1 && (P > 0 || K > 0)) {   // one query: the select may run inside the index launch
-    f.hrows = c.take<uint32_t>((size_t)kFsMaxG * kBuckets);
-    f.red = c.take<uint32_t>(kBuckets);
-    f.stot = c.take<uint32_t>(kFsMaxG);
-    f.cnts = c.take<uint32_t>((size_t)kFsMaxG * 8);
-    f.tkeys = c.take<uint64_t>((size_t)kFsMaxG * 2 * kFsOwnCap);
-    // the counts that must start at zero live in the region zeroed for the
-    // top-k anyway: the digit counts in the (then unused) histogram, the
-    // barrier in the select header
-    f.radix = t.hist;
-    f.bar = t.sel_hdr;
-  }
   if (scores) *scores = sc;
   if (ts) *ts = t;
-  if (fs) *fs = f;
   return c.used + 256;
 }
 
@@ -156,7 +141,7 @@ int32_t csa2_trace_attach(void* table) {
 
 size_t csa2_index_full_workspace(int32_t nq, int32_t max_ctx, int32_t P, int32_t K) {
   if (nq < 1 || max_ctx < 1) return 0;
-  return index_full_ws(nq, max_ctx, P, K, nullptr, nullptr, nullptr, nullptr);
+  return index_full_ws(nq, max_ctx, P, K, nullptr, nullptr, nullptr);
 }
 
 int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
@@ -179,32 +164,13 @@ int32_t csa2_index_full(const int8_t* q, const int8_t* w, const csa2_rows* keys,
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int32_t* sc_ws;
   TopkScratch ts;
-  FusedSel fs;
-  index_full_ws(nq, max_ctx, P, K, ws, &sc_ws, &ts, &fs);
+  index_full_ws(nq, max_ctx, P, K, ws, &sc_ws, &ts);
   int32_t* sc = scores ? scores : sc_ws;
   const int64_t ld = scores ? ld_scores : max_ctx;
   const bool topk = P > 0 || K > 0;
   if (topk && !launch_opts().prezeroed) {
     cudaError_t e = cudaMemsetAsync(ts.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return CSA2_ERR_CUDA;
-  }
-  if (topk && nq == 1) {   // one query: pool and selection inside the index launch when it fits
-    fs.on = 1;
-    fs.n_k = 0;
-    if (P > 0) {
-      fs.k[fs.n_k] = P;
-      fs.out_idx[fs.n_k] = pool_idx;
-      fs.out_cnt[fs.n_k++] = pool_cnt;
-    }
-    if (K > 0) {
-      fs.k[fs.n_k] = K;
-      fs.out_idx[fs.n_k] = sel_idx;
-      fs.out_cnt[fs.n_k++] = sel_cnt;
-    }
-    cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,
-                                       nullptr, status, st, nullptr, &fs);
-    if (e != cudaErrorNotSupported) return cuda_status(e);
-    (void)cudaGetLastError();
   }
   bool hist_built = false;
   cudaError_t e = launch_index_score(q, w, *keys, seq_of_query, query_pos, nq, H, D, max_ctx, sc, ld,
@@ -449,12 +415,13 @@ int32_t csa2_layer_plan(const int32_t* modes, int32_t L, const csa2_layer* layer
   }
   LaunchOpts opts;
   opts.group = s->group_queries != 0;
+  opts.plan = true;
   if (n_full == 1 && n_reindex <= kMaxReindexJobs) {
     void* zp[3];
     size_t zb[3];
     int nz = 0;
     TopkScratch ts;
-    index_full_ws(s->nq, s->max_ctx, s->P, s->K, p.index_base, nullptr, &ts, nullptr);
+    index_full_ws(s->nq, s->max_ctx, s->P, s->K, p.index_base, nullptr, &ts);
     zp[nz] = ts.hist;
     zb[nz++] = topk_zero_bytes(s->nq);
     if (n_reindex > 0) {

@@ -21,7 +21,6 @@
 // Work is the flat list of (query, 128-row tile) items over all queries,
 // split evenly between CTAs, so ragged batches stay balanced.
 #include "csa2_device.cuh"
-#include "fused_select.cuh"
 #include "internal.h"
 
 namespace csa2 {
@@ -41,7 +40,6 @@ struct IndexArgs {
   int64_t ld;
   uint32_t* hist;
   int32_t* status;
-  FusedSel fs;   // fs.on: one query's pool and selection in the same launch
 };
 
 constexpr int kMaxQueries = 4096;   // per launch (the work list prefix lives in shared memory)
@@ -53,8 +51,16 @@ struct IndexCfg {
   static constexpr int kStages = (D == 128) ? 8 : 12;         // >= 96 KiB in flight per SM
 };
 
-constexpr int kEpiThreads = 256;   // 8 epilogue warps: two groups, one warp per TMEM lane quarter each
-__device__ __forceinline__ void named_sync_epi() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Epilogue warps.  One query per segment: 8, two groups of four (one warp per
+// TMEM lane quarter) on alternate tiles.  Queries sharing tiles: 16, four per
+// lane quarter, warp group m reading query m of every tile, so that four
+// warps per scheduler hide the TMEM and arithmetic latencies.
+template <int QG>
+constexpr int epi_warps() { return QG == 1 ? 8 : 16; }
+template <int QG>
+__device__ __forceinline__ void named_sync_epi() {
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * epi_warps<QG>()) : "memory");
+}
 
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_ns();
@@ -67,13 +73,15 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
 // QG queries of one sequence share each key tile (QG = 1 for decode; 4 for a
 // prefill chunk, where consecutive queries of a sequence form the groups).
 template <int D, int N, int QG>
-__global__ void __launch_bounds__(64 + kEpiThreads, 1)
+__global__ void __launch_bounds__(64 + 32 * epi_warps<QG>(), 1)
 index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) {
+  constexpr int kEpiThreads = 32 * epi_warps<QG>();
   using Cfg = IndexCfg<D>;
   constexpr int NST = Cfg::kStages;
   constexpr int TILE = Cfg::kTile;
   constexpr int NG = N * QG;            // MMA N: the heads of every query of a group
   static_assert(NG <= 256, "one MMA covers the group");
+  static_assert(QG == 1 || QG == epi_warps<QG>() / 4, "grouped epilogue: one warp group of four per query of the group");
   // As many TMEM accumulator buffers as fit in the 512 columns (at most 8),
   // so the MMA can run up to NBUF tiles ahead of the epilogue.
   constexpr int NBUF = (512 / NG) < 8 ? (512 / NG) : 8;
@@ -105,10 +113,9 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int lane = tid & 31;
   // trace points: 1 prologue done, 2 first TMA issued, 3 first stage landed,
   // 4 first epilogue tile done, 5 last epilogue tile done, 6 histogram
-  // flushed, 7 producer done, 8 MMA issuer done, 9 stream done, 10 pool and
-  // selection written, and inside the fused select: 11 rows stored, 12 slices
-  // summed, 13 thresholds, 14 counts published, 15 ties resolved
+  // flushed, 7 producer done, 8 MMA issuer done, 9 exit
   CSA2_TRACE_BEGIN(kTrIndex, tid == 0);
+  if (tid == 0) prefetch_tensormap(&kmap);   // the descriptor's fetch overlaps the prologue
 
   // ---- prologue: warp 0 builds the work list (groups of queries and the
   // tiles before each group), warp 1 allocates TMEM, thread 0 sets up the
@@ -121,13 +128,11 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     }
     for (int i = 0; i < NBUF; ++i) {
       mbar_init(&tfull[i], 1);
-      mbar_init(&tempty[i], kEpiThreads / 64);   // one arrival per warp of the group that reads it
+      // one arrival per warp that reads the buffer: a group of four, or every epilogue warp
+      mbar_init(&tempty[i], QG == 1 ? 4 : epi_warps<QG>());
     }
     mbar_init(bready, kEpiThreads / 32);
-    for (int k = 0; k < QG; ++k) {
-      bound_acc[k] = 0ull;
-      mpos[k] = -1;   // a CTA with no segment (no valid position) keeps -1
-    }
+    for (int k = 0; k < QG; ++k) bound_acc[k] = 0ull;
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -204,7 +209,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   pdl_trigger();   // the next grid may be launched (it waits for this one to finish)
   if (warp >= 2) {   // the epilogue's histogram, zeroed before its first use
     for (int i = tid - 64; i < kHist; i += kEpiThreads) hist_s[i] = 0;
-    named_sync_epi();
+    named_sync_epi<QG>();
   }
 
   const int64_t total = prefix[ngroups];
@@ -225,8 +230,8 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   // Between segments the whole CTA synchronises, so the B operand (the
   // queries) and the histogram can be swapped without any hand-off protocol.
   // `git` numbers the items of the CTA and drives every barrier phase.
-  const int et = tid - 64;                 // epilogue thread 0..255 (negative for warps 0-1)
-  const int group = et >> 7;               // epilogue group: tiles i with i % 2 == group
+  const int et = tid - 64;                 // epilogue thread 0..kEpiThreads-1 (negative for warps 0-1)
+  const int group = et >> 7;               // warp group of four: tiles i % 2 (QG 1) or query `group` (QG 4)
   const int quarter = warp & 3;            // TMEM lanes this warp may access
   const int row = quarter * 32 + lane;     // key row of the tile this thread owns
   int64_t git = 0;
@@ -266,7 +271,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       fence_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bready);
-      named_sync_epi();
+      named_sync_epi<QG>();
       for (int r = et; r < nm * a.H; r += kEpiThreads) {
         const int k = r / a.H, h = r % a.H;
         int32_t sq = 0;
@@ -369,7 +374,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
 #pragma unroll
         for (int h = 0; h < N; ++h) wreg[h] = w_s[h];
       }
-      for (int i = group; i < n_it; i += 2) {
+      for (int i = QG == 1 ? group : 0; i < n_it; i += QG == 1 ? 2 : 1) {
         const int64_t gi = git + i;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[gi % NBUF], (uint32_t)((gi / NBUF) & 1), abort_flag));
         const int32_t pos = (tile0 + i) * 128 + row;
@@ -401,55 +406,37 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
             }
           }
         } else {
-          // The group's N-column blocks (query k, head chunk c) are read 32 (or
-          // N) columns at a time, each load issued before the arithmetic of the
-          // block before it, so the TMEM latency overlaps the sums.
-          constexpr int CH = N < 32 ? N : 32;        // columns per block
-          constexpr int NCH = N / CH;                // blocks per query
-          const int nblk = nm * NCH;
-          uint32_t rb[2][CH];
-          auto ld_blk = [&](int bi, uint32_t (&dst)[CH]) {
-            const uint32_t ta = tbase + (uint32_t)((bi / NCH) * N + (bi % NCH) * CH);
-            if constexpr (CH == 16) tmem_ld16(ta, dst);
-            else tmem_ld32(ta, dst);
-          };
-          if (ok) {
-            ld_blk(0, rb[0]);
-            tmem_wait_ld();
-          }
-          int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-#pragma unroll 1
-          for (int bi = 0; bi < nblk; bi += 2) {
+          // Warp group m reads query m of the tile: its N head dots, 32 (or N)
+          // columns at a time, and the head weights 8 at a time; every warp
+          // frees the buffer once, after its last TMEM read.
+          constexpr int CH = N < 32 ? N : 32;
+          const int k = group;
+          int32_t sc = 0;
+          if (ok && k < nm) {
+            int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
-            for (int hb = 0; hb < 2; ++hb) {   // block bi + hb sits in rb[hb]
-              const int cur = bi + hb;
-              if (cur < nblk) {
-                if (ok && cur + 1 < nblk) ld_blk(cur + 1, rb[hb ^ 1]);
-                if (cur + 1 == nblk) {   // the buffer's last block is in registers: free it
-                  tc_fence_before();
-                  __syncwarp();
-                  if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
-                }
-                const int k = cur / NCH, c0 = (cur % NCH) * CH;
-                int4 wv[CH / 4];
+            for (int c = 0; c < N / CH; ++c) {
+              uint32_t rb[CH];
+              if constexpr (CH == 16) tmem_ld16(tbase + (uint32_t)(k * N + c * CH), rb);
+              else tmem_ld32(tbase + (uint32_t)(k * N + c * CH), rb);
+              tmem_wait_ld();
 #pragma unroll
-                for (int u = 0; u < CH / 4; ++u) wv[u] = reinterpret_cast<const int4*>(w_s + k * N + c0)[u];
-                const int32_t* wp = reinterpret_cast<const int32_t*>(wv);
+              for (int h8 = 0; h8 < CH; h8 += 8) {
+                const int4 w0 = *reinterpret_cast<const int4*>(w_s + k * N + c * CH + h8);
+                const int4 w1 = *reinterpret_cast<const int4*>(w_s + k * N + c * CH + h8 + 4);
+                const int32_t wp[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                for (int h = 0; h < CH; ++h) part[h & 7] += wp[h] * max((int32_t)rb[hb][h], 0);
-                if (c0 + CH == N) {   // query k is complete
-                  const int32_t sc =
-                      ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-#pragma unroll
-                  for (int z = 0; z < 8; ++z) part[z] = 0;
-                  if (ok && pos <= mpos[k]) a.scores[(int64_t)(q0 + k) * a.ld + pos] = sc;
-                }
-                if (ok && cur + 1 < nblk) tmem_wait_ld();
+                for (int j = 0; j < 8; ++j) part[j] += wp[j] * max((int32_t)rb[h8 + j], 0);
               }
             }
+            sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
+          if (ok && k < nm && pos <= mpos[k]) a.scores[(int64_t)(q0 + k) * a.ld + pos] = sc;
         }
-        if (nm == 0) {   // no query (cannot happen for a segment with tiles): still free the buffer
+        if (QG == 1 && nm == 0) {   // no query (cannot happen for a segment with tiles): still free the buffer
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&tempty[gi % NBUF]);
@@ -458,7 +445,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       }
       CSA2_MARK(kTrIndex, 5, tid == 64);
       // this query's histogram goes to global memory
-      named_sync_epi();
+      named_sync_epi<QG>();
       if constexpr (QG == 1) {
         if (a.hist) {
           for (int b2 = et; b2 < kBuckets; b2 += kEpiThreads) {
@@ -490,20 +477,6 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   CSA2_MARK(kTrIndex, 9, tid == 0);
   if (warp == 1) tmem_dealloc(tmem_base, TMEM_COLS);
   if (tid == 0 && *abort_flag) record_error(a.status, CSA2_ERR_TIMEOUT);
-  if constexpr (QG == 1) {
-    if (a.fs.on) {   // one query, one CTA per SM: the pool and selection here, after the stream
-      // this CTA's positions: its tiles [lo, hi) of the query's single group, up to the query position
-      const int32_t qp = mpos[0];
-      const int64_t p_hi64 = hi * 128 < (int64_t)qp + 1 ? hi * 128 : (int64_t)qp + 1;
-      auto mark = [&](int p) {
-        (void)p;
-        CSA2_MARK(kTrIndex, p, tid == 0);
-      };
-      fused_select<64 + kEpiThreads, (NST * TILE - kFsGather * 8) / 4>(
-          a.fs, a.scores, hist_s, stages, (int32_t)(lo * 128), (int32_t)(p_hi64 > 0 ? p_hi64 : 0), a.status, mark);
-      CSA2_MARK(kTrIndex, 10, tid == 0);
-    }
-  }
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -541,7 +514,7 @@ cudaError_t launch_one(const CUtensorMap& map, const IndexArgs& a, int grid, cud
   static SetupMask done{0};
   cudaError_t e = ensure_smem(index_score_kernel<D, N, QG>, (int)index_smem_bytes<D>(N, QG, kMaxQueries), done);
   if (e != cudaSuccess) return e;
-  return launch_k(index_score_kernel<D, N, QG>, dim3(grid), dim3(64 + kEpiThreads), smem, st, false,
+  return launch_k(index_score_kernel<D, N, QG>, dim3(grid), dim3(64 + 32 * epi_warps<QG>()), smem, st, false,
                   launch_opts().pdl, map, a);
 }
 
@@ -553,22 +526,11 @@ int sm_count() {
   return n;
 }
 
-// Whether one query's pool and selection can run inside its index-score
-// launch: every CTA's positions fit in its freed key ring, and the scratch
-// covers the CTA count.
-bool fused_select_fits(int32_t D, int32_t max_ctx, int grid) {
-  const int64_t tiles = (max_ctx + 127) / 128;
-  const int64_t per_cta = (tiles + grid - 1) / grid * 128;
-  const int64_t maxp = D == 128 ? (IndexCfg<128>::kStages * IndexCfg<128>::kTile - kFsGather * 8) / 4
-                                : (IndexCfg<64>::kStages * IndexCfg<64>::kTile - kFsGather * 8) / 4;
-  return grid >= 1 && grid <= kFsMaxG && per_cta <= maxp;
-}
-
 cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st, bool* hist_built, const FusedSel* fs) {
+                               cudaStream_t st, bool* hist_built) {
   if (nq > kMaxQueries) return cudaErrorInvalidValue;
   EncodeTiledFn enc = encode_fn();
   if (!enc) return cudaErrorNotSupported;
@@ -586,19 +548,16 @@ cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows
   const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
   // Many queries (a prefill chunk) share key tiles in groups of four, with the
   // histogram left to the top-k; decode keeps one query per segment.  A plan
-  // call that says its queries come in same-sequence blocks (a verify block)
-  // groups them from two queries on.
-  const bool grouped = N <= 64 && (nq >= kGroupMinQueries || (launch_opts().group && nq >= 2));
+  // call groups only when it says its queries come in same-sequence blocks (a
+  // verify block), and then from two queries on; a plan's batch of distinct
+  // sequences keeps one query per segment whatever its size.
+  const LaunchOpts& lo = launch_opts();
+  const bool grouped = N <= 64 && (lo.group ? nq >= 2 : (!lo.plan && nq >= kGroupMinQueries));
   if (hist_built) *hist_built = !grouped && hist;
   IndexArgs a{q, w, seq_of_query, query_pos, to_rowmap(keys), nq, H, max_ctx, scores, ld,
-              grouped ? nullptr : hist, status, FusedSel{}};
+              grouped ? nullptr : hist, status};
   const int64_t upper = (int64_t)nq * ((max_ctx + 127) / 128);
   const int grid = (int)(upper < sm_count() ? (upper > 0 ? upper : 1) : sm_count());
-  if (fs && fs->on) {
-    if (grouped || nq != 1 || !fused_select_fits(D, max_ctx, grid)) return cudaErrorNotSupported;
-    a.fs = *fs;
-    a.hist = nullptr;   // the histogram stays in each CTA's shared memory
-  }
   if (D == 128) {
     switch (N) {
       case 16: return grouped ? launch_one<128, 16, 4>(map, a, grid, st) : launch_one<128, 16, 1>(map, a, grid, st);

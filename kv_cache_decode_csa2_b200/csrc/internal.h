@@ -50,11 +50,15 @@ struct Carver {
 //   prezeroed  the top-k, reindex and attention scratch was zeroed by the
 //              caller (in the kernel launched just before);
 //   group      index scans group the queries of a sequence from 2 queries on
-//              (a verify block), not only from 16.
+//              (a verify block), not only from 16;
+//   plan       the call comes from a layer plan: its index scans group queries
+//              only when `group` says so (a decode batch of distinct sequences
+//              keeps one query per segment and the fused histogram).
 struct LaunchOpts {
   bool pdl = false;
   bool prezeroed = false;
   bool group = false;
+  bool plan = false;
 };
 LaunchOpts& launch_opts();
 struct LaunchOptsScope {   // sets the options for its lifetime
@@ -125,16 +129,11 @@ TopkScratch carve_topk(Carver& c, int32_t nq, int32_t n_max);
 // K1: scores of every visible position for every query (tcgen05 int8), plus
 // the bucket histogram.  hist may be NULL.  *hist_built (if given) says
 // whether the histogram was built: launches of many queries leave it out.
-// With fs (fs->on), one query's pool and selection run in the same launch
-// after the stream (fused_select.cuh); returns cudaErrorNotSupported, having
-// queued nothing, when that does not fit (see fused_select_fits).
-struct FusedSel;
 cudaError_t launch_index_score(const int8_t* q, const int8_t* w, const csa2_rows& keys,
                                const int32_t* seq_of_query, const int32_t* query_pos,
                                int32_t nq, int32_t H, int32_t D, int32_t max_ctx,
                                int32_t* scores, int64_t ld, uint32_t* hist, int32_t* status,
-                               cudaStream_t st, bool* hist_built = nullptr, const FusedSel* fs = nullptr);
-bool fused_select_fits(int32_t D, int32_t max_ctx, int grid);
+                               cudaStream_t st, bool* hist_built = nullptr);
 
 // Radix top-k over score rows.  ks[0..n_k) are the wanted counts (n_k <= 2,
 // ks[0] >= ks[1]); outputs go to out_idx[t]/out_cnt[t].  If hist_ready, the

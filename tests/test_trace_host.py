@@ -48,7 +48,7 @@ def test_summary_times_from_a_known_table():
     assert z.ctas == 1 and z.start_us == 0.0 and abs(z.end_us - 1.0) < 1e-9
     assert k1.ctas == 2 and abs(k1.start_us - 2.0) < 1e-9 and abs(k1.end_us - 23.0) < 1e-9
     names = [p.name for p in k1.points]
-    assert names == ["entry", "prologue done", "stream done"]
+    assert names == ["entry", "prologue done", "exit"]
     entry, pro, ext = k1.points
     assert abs(entry.median_us - 2.5) < 1e-9 and abs(entry.max_us - 3.0) < 1e-9
     assert abs(pro.median_us - 3.5) < 1e-9 and abs(pro.max_us - 4.5) < 1e-9 and pro.reached == 2

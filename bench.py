@@ -85,7 +85,7 @@ QUANT_SAMPLE_ROWS = 65536
 # DRAM bytes (read + write) of one index-score launch on the 1M decode
 # workload, from one ncu capture of this kernel (its summary is kept with the
 # profiles); None when that kernel changed after the capture.
-K1_TRAFFIC_BYTES = {"decode": 134_273_792 + 4_593_664}
+K1_TRAFFIC_BYTES: dict = {}
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 NOMINAL_HBM_GBS = 8000.0
 REPEATS = 5

@@ -96,7 +96,8 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   int32_t* w_s = reinterpret_cast<int32_t*>(hist_s + kHist);     // [NG] (at least 128)
   int32_t* prefix = w_s + (NG > 128 ? NG : 128);                 // [groups + 1] tiles before each group
   int32_t* gq = prefix + ((a.nq + 2) & ~1);                      // [groups + 1] first query of each group
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gq + ((a.nq + 2) & ~1));
+  int32_t* gseq = gq + ((a.nq + 2) & ~1);                        // [groups] sequence of each group
+  uint64_t* bars = reinterpret_cast<uint64_t*>(gseq + ((a.nq + 2) & ~1));
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
   uint64_t* tfull = bars + 2 * NST;
@@ -117,8 +118,8 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   CSA2_TRACE_BEGIN(kTrIndex, tid == 0);
   if (tid == 0) prefetch_tensormap(&kmap);   // the descriptor's fetch overlaps the prologue
 
-  // ---- prologue: warp 0 builds the work list (groups of queries and the
-  // tiles before each group), warp 1 allocates TMEM, thread 0 sets up the
+  // ---- prologue: warp 0 builds the work list (groups of queries, their
+  // sequences and the tiles before each group), warp 1 allocates TMEM, thread 0 sets up the
   // barriers; one block barrier later the producer streams.  The epilogue
   // warps zero their histogram behind a barrier of their own.
   if (tid == 0) {
@@ -185,6 +186,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       const int g = base + lane;
       int32_t v = 0;
       if (g < n_groups) {
+        gseq[g] = a.seq_of_query ? __ldg(a.seq_of_query + gq[g]) : gq[g];   // in flight with the positions
         for (int i = gq[g]; i < gq[g + 1]; ++i) {
           const int32_t pos = __ldg(a.query_pos + i);
           if (pos < 0 || pos >= a.max_ctx) record_error(a.status, CSA2_ERR_INDEX_RANGE);
@@ -291,36 +293,68 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
 
     if (warp == 0) {
       // ---------------------------------------------------------- producer
-      if (lane == 0) {
-        prefetch_tensormap(&kmap);
-        const uint64_t pol = l2_policy_evict_first();
-        const int32_t seq = a.seq_of_query ? __ldg(a.seq_of_query + q0) : q0;
-        int i = 0;
-        for (; i < n_it; ++i) {
+      // Lane 0 issues the loads.  With a paged view the whole warp reads the
+      // page-table entries one chunk of 16 tiles ahead (lane l: box l & 1 of
+      // tile l >> 1 of the chunk), so no load waits on a table lookup.
+      const uint64_t pol = l2_policy_evict_first();
+      const int32_t seq = gseq[g];
+      const RowMap& m = a.rows;
+      auto page_entry = [&](int i0) -> int32_t {   // raw entry behind this lane's box of the chunk at i0
+        const int i = i0 + (lane >> 1);
+        const int32_t p0 = (tile0 + i) * 128 + 64 * (lane & 1);
+        if (i >= n_it || p0 > pos_hi) return -1;
+        const int32_t pg = p0 / m.page_rows;
+        return pg < m.max_pages ? __ldg(m.page_table + (int64_t)seq * m.max_pages + pg) : -1;
+      };
+      int32_t ent = -1, ent_next = -1;
+      if (m.page_table) {
+        ent = page_entry(0);
+        ent_next = page_entry(16);
+      }
+      int i = 0;
+      for (; i < n_it; ++i) {
+        if (m.page_table && i > 0 && i % 16 == 0) {
+          ent = ent_next;
+          ent_next = page_entry(i + 16);
+        }
+        const int32_t tile = tile0 + i;
+        int64_t r[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int32_t p0 = tile * 128 + 64 * j;
+          if (m.page_table) {
+            const int32_t e = __shfl_sync(0xffffffffu, ent, 2 * (i % 16) + j);
+            const int64_t row = (int64_t)e * m.page_rows + (p0 % m.page_rows);
+            r[j] = (e >= 0 && row < m.n_rows) ? row : -1;
+          } else {
+            r[j] = map_row(m, seq, p0);
+          }
+          if (p0 > pos_hi) r[j] = -2;   // past the last visible position: no box
+        }
+        bool ok = true;
+        if (lane == 0) {
           const int64_t gi = git + i;
           const int st = (int)(gi % NST);
           const uint32_t ph = (uint32_t)((gi / NST) & 1);
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) break;
-          const int32_t tile = tile0 + i;
-          int64_t r[2];
-          uint32_t bytes = 0;
+          ok = mbar_wait(&empty[st], ph ^ 1, abort_flag);
+          if (ok) {
+            uint32_t bytes = 0;
 #pragma unroll
-          for (int j = 0; j < 2; ++j) {
-            const int32_t p0 = tile * 128 + 64 * j;
-            r[j] = -1;
-            if (p0 <= pos_hi) {
-              r[j] = map_row(a.rows, seq, p0);
-              if (r[j] < 0) record_error(a.status, CSA2_ERR_INDEX_RANGE);
-              else bytes += 64 * D;
+            for (int j = 0; j < 2; ++j) {
+              if (r[j] == -1) record_error(a.status, CSA2_ERR_INDEX_RANGE);
+              else if (r[j] >= 0) bytes += 64 * D;
             }
-          }
-          mbar_arrive_expect_tx(&full[st], bytes);
+            mbar_arrive_expect_tx(&full[st], bytes);
 #pragma unroll
-          for (int j = 0; j < 2; ++j)
-            if (r[j] >= 0)
-              tma_load_2d(stages + st * TILE + j * 64 * D, &kmap, 0, (int32_t)r[j], &full[st], pol);
-          CSA2_MARK(kTrIndex, 2, gi == 0);
+            for (int j = 0; j < 2; ++j)
+              if (r[j] >= 0)
+                tma_load_2d(stages + st * TILE + j * 64 * D, &kmap, 0, (int32_t)r[j], &full[st], pol);
+            CSA2_MARK(kTrIndex, 2, gi == 0);
+          }
         }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      }
+      if (lane == 0) {
         if (*abort_flag) {   // let loads already in flight land before moving on
           const int64_t issued = git + i;
           const int64_t n = i < NST ? i : NST;
@@ -448,11 +482,20 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       named_sync_epi<QG>();
       if constexpr (QG == 1) {
         if (a.hist) {
-          for (int b2 = et; b2 < kBuckets; b2 += kEpiThreads) {
-            const uint32_t v = hist_s[b2];
-            if (v) {
-              atomicAdd(a.hist + (int64_t)q0 * kBuckets + b2, v);
-              hist_s[b2] = 0;
+          // Four bins per 16-byte read; each populated pair of bins costs one
+          // 64-bit add (a count never reaches 2^32, so the low bin cannot
+          // carry into the high one, and the pair is the two 32-bit bins in
+          // memory order).  The adds of every CTA meet in a few L2 slices at
+          // the end of the launch, and the next grid waits for all of them:
+          // their number, not their size, sets that wait.
+          unsigned long long* gh = reinterpret_cast<unsigned long long*>(a.hist + (int64_t)q0 * kBuckets);
+          for (int b4 = et; b4 < kBuckets / 4; b4 += kEpiThreads) {
+            uint4* hp = reinterpret_cast<uint4*>(hist_s) + b4;
+            const uint4 v = *hp;
+            if (v.x | v.y | v.z | v.w) {
+              if (v.x | v.y) atomicAdd(gh + 2 * b4, (unsigned long long)v.x | ((unsigned long long)v.y << 32));
+              if (v.z | v.w) atomicAdd(gh + 2 * b4 + 1, (unsigned long long)v.z | ((unsigned long long)v.w << 32));
+              *hp = make_uint4(0, 0, 0, 0);
             }
           }
         }
@@ -504,7 +547,7 @@ size_t index_smem_bytes(int N, int QG, int nq) {
   using Cfg = IndexCfg<D>;
   const int NG = N * QG;
   return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)NG * D + (QG == 1 ? kBuckets * 4 : 0) +
-         (size_t)(NG > 128 ? NG : 128) * 4 + 2 * (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 +
+         (size_t)(NG > 128 ? NG : 128) * 4 + 3 * (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 +
          32 + 8 * (size_t)QG + 4 * (size_t)QG + 16;
 }
 

@@ -185,7 +185,9 @@ cudaError_t launch_reindex_score(const int8_t* q, const int8_t* w, const csa2_ro
                                  int32_t P, int32_t* scores, int32_t* status, cudaStream_t st);
 
 // K3 fused: scores and top-K of up to kMaxReindexJobs reindex layers that
-// search the same pool, in one launch of co-resident CTAs.
+// search the same pool, in one launch: co-resident CTAs that meet at grid
+// barriers, or, for batches too large to be co-resident with pools of up to
+// kRLastMaxP slots, the last CTA of each pool to finish its scores selects.
 constexpr int kMaxReindexJobs = 8;
 struct ReindexJobDesc {
   const int8_t* q;           // [nq][H][D]
@@ -202,12 +204,14 @@ struct ReindexSelScratch {
   uint64_t* ties;
   uint32_t* mcnt;
   uint32_t* radix;
+  int32_t* sc;               // [n_probs][P] the pool's scores, when the job keeps none
 };
+constexpr int kRLastMaxP = 16384;
 size_t reindex_select_scratch_bytes(int32_t n_probs, int32_t P);
 ReindexSelScratch carve_reindex_select(Carver& c, int32_t n_probs, int32_t P);
-// Returns cudaErrorNotSupported, having queued nothing, when the CTAs cannot
-// be co-resident or the head count is above 64; the caller then scores and
-// selects in separate launches.
+// Returns cudaErrorNotSupported, having queued nothing, when pools above
+// kRLastMaxP slots need more CTAs than can be co-resident, or the head count
+// is above 64; the caller then scores and selects in separate launches.
 cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, const int32_t* seq_of_query,
                                   const int32_t* pool_idx, const int32_t* pool_cnt, int32_t nq, int32_t H,
                                   int32_t D, int32_t P, int32_t K, const ReindexSelScratch& r,

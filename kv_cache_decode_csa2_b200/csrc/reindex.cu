@@ -8,9 +8,11 @@
 // group, D[128 slots x N heads] in TMEM, and applies the ReLU and head-weight
 // epilogue of the full-mode scorer.
 //
-// reindex_select_kernel goes on to the top-K of the layer in the same launch:
-// the CTAs of a pool (every CTA holds 128 of its scores, one per thread) are
-// co-resident and meet at bounded grid barriers.  They build the bucket
+// reindex_select_kernel goes on to the top-K of the layer in the same launch.
+// The CTAs of a pool (every CTA holds 128 of its scores, one per thread) are
+// co-resident and meet at bounded grid barriers; batches of pools too large
+// to be co-resident let the CTA of each pool that finishes its scores last
+// select alone (see LAST below).  They build the bucket
 // histogram of the pool in global memory, find the threshold bucket b*, rank
 // the ties at b* (the pool's tie list, staged in shared memory), and write the
 // members in slot order, which is position order because pool positions
@@ -187,17 +189,21 @@ struct RSelArgs {
   uint64_t* ties;     // [probs][kRTieCap]
   uint32_t* mcnt;     // [probs][G]
   uint32_t* radix;    // [probs][8][256]
+  int32_t* sc;        // [probs][P] scores of pools whose job keeps none (last-CTA select)
   int32_t* status;
 };
 
 // Dynamic shared memory: the T tiles of 128 pool rows and the query (then the
 // pool's ties), w, this CTA's ties, the MMA barrier and the TMEM address.
-template <int D, int N, int T>
+// LAST: the region holds, after scoring, the pool's scores and the padded
+// histogram (then the ties) of the selecting CTA.
+template <int D, int N, int T, bool LAST>
 struct RSelLayout {
   static constexpr int NT = 128 * T;
   static constexpr size_t tiles = (size_t)(T * 128 * D + N * D);
-  static constexpr size_t ties_or_hist = (size_t)kRTieCap * 8 > (size_t)kBuckets * 4 ? (size_t)kRTieCap * 8
-                                                                                      : (size_t)kBuckets * 4;
+  static constexpr size_t ties_or_hist = LAST ? (size_t)kRLastMaxP * 4 + (size_t)(kBuckets + kBuckets / 32) * 4
+                                         : (size_t)kRTieCap * 8 > (size_t)kBuckets * 4 ? (size_t)kRTieCap * 8
+                                                                                        : (size_t)kBuckets * 4;
   static constexpr size_t region = tiles > ties_or_hist ? tiles : ties_or_hist;   // reused after scoring
   static constexpr size_t smem = 1024 + region + 128 * 4 + NT * 8 + 64;
   static constexpr uint32_t cols = T * N <= 32 ? 32 : T * N <= 64 ? 64 : T * N <= 128 ? 128 : 256;
@@ -205,9 +211,20 @@ struct RSelLayout {
 
 // T tiles of 128 pool slots per CTA (one slot per thread): the device holds
 // one such CTA per SM, so T sets how many pools fit in one launch.
-template <int D, int N, int T>
-__global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid_constant__ RSelArgs a) {
-  using Lay = RSelLayout<D, N, T>;
+//
+// LAST: every CTA publishes its scores and counts itself in with one
+// acquire-release add; the CTA that arrives last (it then sees every score of
+// the pool) selects the pool's top-K alone: kRLastE consecutive slots per
+// thread in registers, the bucket histogram in shared memory, the ties at
+// the threshold bucket ranked in shared memory, one block scan for the
+// output slots.  Nothing waits on another CTA, so the grid need not be
+// co-resident, and the CTAs that are not last leave as soon as they have
+// published, which lets the next launch start on their SMs.
+constexpr int kRLastE = 64;                              // slots per thread of the selecting CTA
+constexpr int kRLastHist = kBuckets + kBuckets / 32;     // padded histogram words
+template <int D, int N, int T, bool LAST>
+__global__ void __launch_bounds__(128 * T, LAST ? 2 : 1) reindex_select_kernel(const __grid_constant__ RSelArgs a) {
+  using Lay = RSelLayout<D, N, T, LAST>;
   constexpr int NT = Lay::NT;
   constexpr uint32_t TMEM_COLS = Lay::cols;
   extern __shared__ uint8_t smem_raw[];
@@ -231,8 +248,9 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   const int prob = jb * a.nq + q;
   const int G = a.G;
   // trace points: 1 own inputs staged, 2 grid before done, 3 pool rows
-  // gathered, 4 scored, 5 histogram barrier, 6 threshold bucket, 7 tie
-  // barrier, 8 ties ranked, 9 count barrier, 10 written
+  // gathered, 4 scored, 5 histogram barrier (LAST: scores published), 6
+  // threshold bucket, 7 tie barrier, 8 ties ranked, 9 count barrier, 10
+  // written (LAST: 6, 8 and 10 in the selecting CTA only)
   CSA2_TRACE_BEGIN(kTrReindex, tid == 0);
   if (tid == 0) {
     bstar_s = -1;
@@ -348,6 +366,160 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  if constexpr (LAST) {
+    static_assert(NT * kRLastE >= kRLastMaxP, "the selecting CTA holds a whole pool");
+    int32_t* srow = J.scores ? J.scores + (int64_t)q * a.P : a.sc + (size_t)prob * a.P;
+    uint32_t* hdr = a.hdr + (size_t)prob * 4;
+    if (valid) srow[slot] = s;
+    __shared__ uint32_t last_s;
+    __syncthreads();   // the CTA's scores are stored before thread 0's release
+    if (tid == 0) {
+      uint32_t old;
+      asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(hdr) : "memory");
+      last_s = old == (uint32_t)G - 1u;
+    }
+    __syncthreads();
+    CSA2_MARK(kTrReindex, 5, tid == 0);
+    if (!last_s) return;
+
+    // ---- the last CTA: every score of the pool is visible (thread 0's
+    // acquire, then the block barrier).  Thread t owns the kRLastE slots
+    // j0 = t kRLastE ..; shared memory holds the scores with slot j0 + u at
+    // sc_s[u NT + t] (lanes read consecutive words), then the bucket
+    // histogram with one pad word per 32 bins (bin b at b + b / 32), so that
+    // the thread owning bins 32 t .. 32 t + 31 reads them without conflicts.
+    // Loops stay rolled: this code runs once per pool, from a cold
+    // instruction cache.
+    int32_t* sc_s = reinterpret_cast<int32_t*>(smem);
+    uint32_t* hs = reinterpret_cast<uint32_t*>(smem + kRLastMaxP * 4);
+    for (int i = tid; i < kRLastHist; i += NT) hs[i] = 0u;
+    const int32_t j0 = tid * kRLastE;
+    const int32_t nv = cnt - j0 < 0 ? 0 : (cnt - j0 > kRLastE ? kRLastE : cnt - j0);
+    const uint64_t vm = nv >= 64 ? ~0ull : ((1ull << nv) - 1ull);   // bit u: slot j0 + u is in the pool
+    if ((reinterpret_cast<uintptr_t>(srow) & 15u) == 0 && (a.P & 3) == 0) {
+      int4 v[kRLastE / 4];
+#pragma unroll
+      for (int u = 0; u < kRLastE / 4; ++u)
+        v[u] = j0 + 4 * u < a.P ? __ldcg(reinterpret_cast<const int4*>(srow + j0) + u) : make_int4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < kRLastE / 4; ++u) {
+        sc_s[(4 * u + 0) * NT + tid] = v[u].x;
+        sc_s[(4 * u + 1) * NT + tid] = v[u].y;
+        sc_s[(4 * u + 2) * NT + tid] = v[u].z;
+        sc_s[(4 * u + 3) * NT + tid] = v[u].w;
+      }
+    } else {
+      for (int u = 0; u < kRLastE; ++u) sc_s[u * NT + tid] = j0 + u < a.P ? __ldcg(srow + j0 + u) : 0;
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int u = 0; u < kRLastE; ++u) {
+      if ((vm >> u) & 1ull) {
+        const uint32_t b = score_bucket(sc_s[u * NT + tid]);
+        atomicAdd(&hs[b + (b >> 5)], 1u);
+      }
+    }
+    __syncthreads();
+
+    // threshold bucket b*: the bucket holding the K-th best score
+    static_assert(kBuckets == 32 * NT, "32 bins per thread");
+    const uint32_t* hb = hs + tid * 33;
+    uint32_t hsum = 0;
+#pragma unroll 8
+    for (int b = 0; b < 32; ++b) hsum += hb[b];
+    uint64_t total64;
+    const uint64_t hex = sel_scan<NT>(hsum, wtmp, &total64);
+    const int64_t total = (int64_t)total64;
+    const int64_t above_me = total - (int64_t)hex - hsum;
+    const int32_t K = a.K;
+    if (total > K && above_me < K && above_me + hsum >= K) {
+      int64_t acc = above_me;
+      for (int b = 31; b >= 0; --b) {
+        if (acc + hb[b] >= K) {
+          bstar_s = tid * 32 + b;
+          above_s = (int32_t)acc;
+          break;
+        }
+        acc += hb[b];
+      }
+    }
+    __syncthreads();
+    CSA2_MARK(kTrReindex, 6, tid == 0);
+    const int32_t bstar = bstar_s;   // -1: every slot of the pool is a member
+
+    // classify; the ties at b* go to one list in shared memory (over the histogram)
+    uint64_t above_m = 0ull, tie_m = 0ull;
+    uint64_t* tl = reinterpret_cast<uint64_t*>(hs);
+#pragma unroll 4
+    for (int u = 0; u < kRLastE; ++u) {
+      if ((vm >> u) & 1ull) {
+        const int32_t sc = sc_s[u * NT + tid];
+        const int32_t bk = (int32_t)score_bucket(sc);
+        if (bk > bstar) {
+          above_m |= 1ull << u;
+        } else if (bk == bstar) {
+          tie_m |= 1ull << u;
+          const uint32_t t = atomicAdd(&own_cnt, 1u);
+          if (t < (uint32_t)kRTieCap) tl[t] = cand_key(sc, j0 + u);
+        }
+      }
+    }
+    __syncthreads();
+    if (bstar >= 0) {
+      const uint32_t nt = own_cnt;
+      const int32_t need = K - above_s;
+      if (nt <= (uint32_t)kRTieCap) {   // a tie is in when fewer than `need` ties beat it
+        for (uint32_t i = warp; i < nt; i += NT / 32) {
+          const uint64_t ki = tl[i];
+          uint32_t r = 0;
+          for (uint32_t j = lane; j < nt; j += 32) r += tl[j] > ki;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) r += __shfl_xor_sync(0xffffffffu, r, o);
+          if (lane == 0 && (int32_t)r < need) atomicMin(&kthr_s, (unsigned long long)ki);
+        }
+      } else {   // a flat distribution: the need-th key among every tie of the pool
+        static_assert(sizeof(ListKthSmem) <= (size_t)kRLastHist * 4, "the select's scratch fits the histogram");
+        const uint64_t k0 = tl[0];
+        ListKthSmem& lk = *reinterpret_cast<ListKthSmem*>(hs);   // over the tie list: k0 is read first
+        const uint64_t kth = block_kth<NT>(
+            (uint32_t)cnt, need,
+            [&](uint32_t i) -> uint64_t {
+              const int32_t v = sc_s[(i % kRLastE) * NT + i / kRLastE];
+              return (int32_t)score_bucket(v) == bstar ? cand_key(v, (int32_t)i) : 0ull;
+            },
+            k0, wtmp, lk);
+        if (tid == 0) kthr_s = kth;
+      }
+      __syncthreads();
+    }
+    CSA2_MARK(kTrReindex, 8, tid == 0);
+    uint64_t mem = above_m;
+    if (tie_m) {
+      const uint64_t kthr = kthr_s;
+      for (int u = 0; u < kRLastE; ++u)
+        if (((tie_m >> u) & 1ull) && cand_key(sc_s[u * NT + tid], j0 + u) >= kthr) mem |= 1ull << u;
+    }
+
+    // the members' slots in pool order (= position order), then their positions
+    uint64_t grand;
+    int64_t k = (int64_t)sel_scan<NT>((uint64_t)__popcll(mem), wtmp, &grand);   // ends with a barrier:
+    int32_t* out_s = sc_s;                                                      // the scores are done
+    for (uint64_t m = mem; m; m &= m - 1ull) {
+      if (k < K) out_s[k] = j0 + __ffsll((long long)m) - 1;
+      ++k;
+    }
+    __syncthreads();
+    const int32_t n_out = grand < (uint64_t)K ? (int32_t)grand : K;
+    int32_t* dst = J.sel_idx + (int64_t)q * K;
+#pragma unroll 4
+    for (int32_t i = tid; i < K; i += NT) dst[i] = i < n_out ? __ldg(pidx + out_s[i]) : -1;
+    if (tid == 0) {
+      if (J.sel_cnt) J.sel_cnt[q] = n_out;
+      hdr[0] = 0u;   // every CTA has arrived: the count is ready for the next launch
+    }
+    CSA2_MARK(kTrReindex, 10, tid == 0);
+    return;
+  }
   if (J.scores && valid) J.scores[(int64_t)q * a.P + slot] = s;
 
   // ---- the pool's bucket histogram, then the threshold bucket.  The CTA
@@ -365,9 +537,12 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
     __syncthreads();
     if (valid) atomicAdd(&hs[bk], 1u);
     __syncthreads();
-    for (int i = tid; i < kBuckets; i += NT) {
-      const uint32_t v = hs[i];
-      if (v) atomicAdd(&hist[i], v);
+    // one 64-bit add per populated pair of buckets (no carry: counts stay far below 2^32)
+    for (int i = tid; i < kBuckets / 2; i += NT) {
+      const uint2 v = reinterpret_cast<const uint2*>(hs)[i];
+      if (v.x | v.y)
+        atomicAdd(reinterpret_cast<unsigned long long*>(hist) + i,
+                  (unsigned long long)v.x | ((unsigned long long)v.y << 32));
     }
   }
   uint32_t phase = 0;
@@ -477,41 +652,49 @@ __global__ void __launch_bounds__(128 * T, 1) reindex_select_kernel(const __grid
   CSA2_MARK(kTrReindex, 10, tid == 0);
 }
 
-template <int D, int N, int T>
+template <int D, int N, int T, bool LAST>
 cudaError_t launch_rs_t(const RSelArgs& a_in, int n_jobs, int nq, size_t zero_bytes, cudaStream_t st) {
-  using Lay = RSelLayout<D, N, T>;
+  using Lay = RSelLayout<D, N, T, LAST>;
   constexpr size_t smem = Lay::smem;
   static SetupMask done{0};
   static std::atomic<int> max_ctas[64];   // co-resident CTAs per device (0: not yet known)
-  cudaError_t e = ensure_smem(reindex_select_kernel<D, N, T>, (int)smem, done);
+  cudaError_t e = ensure_smem(reindex_select_kernel<D, N, T, LAST>, (int)smem, done);
   if (e != cudaSuccess) return e;
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev >= 64) return cudaErrorNotSupported;
-  if (!max_ctas[dev]) {
-    int per_sm = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reindex_select_kernel<D, N, T>, Lay::NT, smem);
-    if (e != cudaSuccess) return e;
-    max_ctas[dev] = per_sm * sm_count();
-  }
   RSelArgs a = a_in;
   a.G = (a.P + Lay::NT - 1) / Lay::NT;
-  if ((int64_t)a.G * nq * n_jobs > max_ctas[dev]) return cudaErrorNotSupported;
+  if constexpr (!LAST) {   // the CTAs of a pool meet at grid barriers: all must be resident
+    int dev = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64) return cudaErrorNotSupported;
+    if (!max_ctas[dev]) {
+      int per_sm = 0;
+      e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, reindex_select_kernel<D, N, T, LAST>, Lay::NT,
+                                                        smem);
+      if (e != cudaSuccess) return e;
+      max_ctas[dev] = per_sm * sm_count();
+    }
+    if ((int64_t)a.G * nq * n_jobs > max_ctas[dev]) return cudaErrorNotSupported;
+  }
   if (!launch_opts().prezeroed) {
     e = cudaMemsetAsync(a.hist, 0, zero_bytes, st);   // histograms and barrier headers
     if (e != cudaSuccess) return e;
   }
-  return launch_k(reindex_select_kernel<D, N, T>, dim3(a.G, nq, n_jobs), dim3(Lay::NT), smem, st, false,
+  return launch_k(reindex_select_kernel<D, N, T, LAST>, dim3(a.G, nq, n_jobs), dim3(Lay::NT), smem, st, false,
                   launch_opts().pdl, a);
 }
 
-// Two tiles per CTA when the CTAs fit on the device, else four.
+// Co-resident CTAs of two tiles each when they fit the device.  Otherwise
+// (a batch of many pools) the last-CTA select for pools of up to kRLastMaxP
+// slots, else co-resident CTAs of four tiles.  The grid-barrier path is the
+// faster one when it fits: its selection work is spread over every CTA of
+// the pool, while the last CTA's runs on one SM.
 template <int D, int N>
 cudaError_t launch_rs(const RSelArgs& a, int n_jobs, int nq, size_t zero_bytes, cudaStream_t st) {
-  cudaError_t e = launch_rs_t<D, N, 2>(a, n_jobs, nq, zero_bytes, st);
+  cudaError_t e = launch_rs_t<D, N, 2, false>(a, n_jobs, nq, zero_bytes, st);
   if (e != cudaErrorNotSupported) return e;
-  return launch_rs_t<D, N, 4>(a, n_jobs, nq, zero_bytes, st);
+  if (a.P <= kRLastMaxP && a.K <= kRLastMaxP) return launch_rs_t<D, N, 2, true>(a, n_jobs, nq, zero_bytes, st);
+  return launch_rs_t<D, N, 4, false>(a, n_jobs, nq, zero_bytes, st);
 }
 
 }  // namespace
@@ -555,6 +738,7 @@ ReindexSelScratch carve_reindex_select(Carver& c, int32_t n_probs, int32_t P) {
   r.ties = c.take<uint64_t>((size_t)n_probs * kRTieCap);
   r.mcnt = c.take<uint32_t>((size_t)n_probs * G);
   r.radix = c.take<uint32_t>((size_t)n_probs * 8 * 256);
+  r.sc = c.take<int32_t>((size_t)n_probs * P);
   return r;
 }
 
@@ -581,6 +765,7 @@ cudaError_t launch_reindex_select(const ReindexJobDesc* jobs, int32_t n_jobs, co
   a.ties = r.ties;
   a.mcnt = r.mcnt;
   a.radix = r.radix;
+  a.sc = r.sc;
   a.status = status;
   const int N = H <= 16 ? 16 : H <= 32 ? 32 : H <= 64 ? 64 : 128;
   if (N == 128) return cudaErrorNotSupported;

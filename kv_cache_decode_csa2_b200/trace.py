@@ -36,7 +36,7 @@ POINT_NAMES = {
     1: ("select", ["entry", "grid before done", "threshold buckets", "classified", "first grid barrier",
                    "row ties staged", "ties ranked", "second grid barrier", "written"]),
     2: ("reindex_select", ["entry", "own inputs staged", "grid before done", "pool rows gathered", "scored",
-                           "histogram barrier", "threshold bucket", "tie barrier", "ties ranked",
+                           "published | histogram barrier", "threshold bucket", "tie barrier", "ties ranked",
                            "count barrier", "written"]),
     3: ("sparse_attn", ["entry", "Q staged", "grid before done", "row positions", "rows dequantised", "logits",
                         "softmax", "P V done", "partial written", "group barrier", "merged"]),

@@ -259,12 +259,17 @@ def test_reindex_flat_scores():
     assert np.array_equal(_np(re.sel_idx)[0], ref_sel) and int(_np(re.sel_cnt)[0]) == wl.topk
 
 
-def test_reindex_batch_of_many_queries():
+@pytest.mark.parametrize("flat", [False, True])
+def test_reindex_batch_of_many_queries(flat):
     """Eight queries of a 16384-entry pool: more CTAs than fit on the device at
-    once, so scoring and selection run as separate launches."""
+    once, so the last CTA of each pool to finish its scores selects alone.
+    flat: all-zero reindex keys, every score ties, and the need-th tie key is
+    found by the radix passes over the whole pool."""
     wl = synth.scaled(synth.C3_RAGGED, ragged=(8, 17000, 30000), modes=(synth.FULL, synth.REINDEX), page_rows=0)
     c = G.build(wl)
     full, re = c.layers_dev
+    if flat:
+        re.keys.data.zero_()
     B.check_status(B.csa2_index_full(full.q, full.w, full.keys, c.pos_dev, c.max_ctx, P=wl.pool,
                                      pool_idx=full.pool_idx, pool_cnt=full.pool_cnt, seq_of_query=c.seq_dev))
     B.check_status(B.csa2_reindex(re.q, re.w, re.keys, full.pool_idx, full.pool_cnt, wl.topk, re.sel_idx,
@@ -275,7 +280,10 @@ def test_reindex_batch_of_many_queries():
         q0, w0 = c.host_q[(0, i)]
         _, ref_pool, _ = O.full_index(q0, w0, c.host_keys[(0, s)], int(c.query_pos[i]), wl.pool, wl.topk)
         q1, w1 = c.host_q[(1, i)]
-        _, ref_sel = O.reindex(q1, w1, c.host_keys[(1, s)], ref_pool, wl.topk)
+        k1 = np.zeros_like(c.host_keys[(1, s)]) if flat else c.host_keys[(1, s)]
+        _, ref_sel = O.reindex(q1, w1, k1, ref_pool, wl.topk)
+        if flat:
+            assert np.array_equal(ref_sel, ref_pool[:wl.topk])
         assert np.array_equal(pools[i, :len(ref_pool)], ref_pool)
         assert np.array_equal(sels[i, :len(ref_sel)], ref_sel)
 

@@ -85,7 +85,10 @@ QUANT_SAMPLE_ROWS = 65536
 # DRAM bytes (read + write) of one index-score launch on the 1M decode
 # workload, from one ncu capture of this kernel (its summary is kept with the
 # profiles); None when that kernel changed after the capture.
-K1_TRAFFIC_BYTES: dict = {}
+K1_TRAFFIC_BYTES = {"decode": 134_281_728 + 3_837_440}
+# DRAM bytes (read + write) of one FP4 cache-write launch of 1,048,576 bf16
+# rows of d512, from one ncu capture (summary kept with the profiles).
+QUANT_TRAFFIC_BYTES = 1_073_840_384 + 268_985_856
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
 NOMINAL_HBM_GBS = 8000.0
 REPEATS = 5
@@ -918,7 +921,7 @@ def run_quantize(args, rank, world, local):
             "roofline": {"kernel": "fp4_quantize_kernel<bf16>", "bound": "hbm", "achieved": achieved,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": achieved / pk["hbm_gbs"],
                          "peak_src": pk["src"], "ms_per_launch": ms, "bytes_per_launch": n * per_row,
-                         "traffic": None},
+                         "traffic": QUANT_TRAFFIC_BYTES if n == 1 << 20 and D == 512 else None},
             "e2e": {"value": world * n / (e_ms / 1e3), "unit": "rows/s",
                     "h2d_bytes_per_step": xh.numel() * xh.element_size(),
                     "d2h_bytes_per_step": ch.numel() + sh.numel(),

@@ -6,11 +6,20 @@
 //   scale = E4M3 nearest to amax/6 (ties to even, saturating at 448)
 //   code  = E2M1 nearest to x/scale (ties to even, saturating at +-6)
 //
-// Both roundings are decided by exact comparisons.  |x| (fp32) is compared
-// with a product of an E2M1 midpoint (at most 3 significant bits) and the
-// scale (4 bits), and amax with 3 * (v_c + v_{c+1}) for adjacent E4M3 values
-// (at most 8 bits).  Every such product is exact in fp32, so no division
-// rounds.  The result is the nearest code of the exact quotient.
+// The scale: the E4M3 code read off amax/6's exponent and top mantissa bits,
+// moved to the largest c with 6 v(c) <= amax by exact comparisons, then the
+// nearest of c and c+1 decided against 3 (v(c) + v(c+1)), an exact product.
+//
+// The codes: q = x/scale from one multiply by the reciprocal and two fused
+// corrections (the residual x - q s is exact, so q is within half an ulp of
+// the quotient plus a term 2^-24 below it, and an exact midpoint stays
+// exact), then sm_100's E2M1 conversion (round to nearest, ties to even,
+// saturating), two values per instruction.  A quotient that is not a
+// midpoint can still round onto one only if the value carries more than 8
+// significant bits: for bf16 input it is at least 2^-8 (relative) away from
+// every midpoint, for fp32 input a q that lands exactly on a midpoint is
+// moved one ulp toward the side the exact residual x - m s gives.  A result
+// of magnitude zero is stored as +0.
 //
 // The input is fp32 or bf16 rows (bf16 widens to fp32 exactly, so both give
 // the codes of the same values).
@@ -29,32 +38,57 @@ __device__ __forceinline__ float e4m3_pos(uint32_t c) {
 
 __device__ __forceinline__ uint32_t e4m3_scale_for(float amax) {
   if (amax >= 6.0f * 448.0f) return 0x7Eu;
-  // largest c with 6*v(c) <= amax (v is increasing in c)
-  uint32_t lo = 0, hi = 126;
-  while (lo < hi) {
-    const uint32_t mid = (lo + hi + 1) >> 1;
-    if (6.0f * e4m3_pos(mid) <= amax) lo = mid; else hi = mid - 1;
+  // a first guess from amax / 6 (approximate), then the exact largest c with 6 v(c) <= amax
+  const float y = amax * (1.0f / 6.0f);
+  int c;
+  if (y < 0.015625f) {   // below the smallest normal 2^-6: v = m 2^-9
+    c = (int)(y * 512.0f);
+  } else {
+    const uint32_t bits = __float_as_uint(y);
+    c = (int)((((bits >> 23) - 120u) << 3) | ((bits >> 20) & 7u));
   }
-  const uint32_t c = lo;
-  if (c == 126u) return c;
-  const float mid2 = 3.0f * (e4m3_pos(c) + e4m3_pos(c + 1));   // 6 * midpoint, exact
-  if (amax > mid2) return c + 1;
-  if (amax < mid2) return c;
-  return (c & 1u) ? c + 1 : c;
+  c = c < 0 ? 0 : (c > 126 ? 126 : c);
+  while (c < 126 && 6.0f * e4m3_pos((uint32_t)c + 1) <= amax) ++c;
+  while (c > 0 && 6.0f * e4m3_pos((uint32_t)c) > amax) --c;
+  if (c == 126) return 126u;
+  const float mid2 = 3.0f * (e4m3_pos((uint32_t)c) + e4m3_pos((uint32_t)c + 1));   // 6 * midpoint, exact
+  if (amax > mid2) return (uint32_t)c + 1;
+  if (amax < mid2) return (uint32_t)c;
+  return (c & 1) ? (uint32_t)c + 1 : (uint32_t)c;
 }
 
-__device__ __forceinline__ uint32_t e2m1_code(float x, float s) {
-  const float ax = fabsf(x);
-  // midpoints between magnitudes 0,.5,1,1.5,2,3,4,6
-  const float mids[7] = {0.25f, 0.75f, 1.25f, 1.75f, 2.5f, 3.5f, 5.0f};
-  uint32_t idx = 0;
-#pragma unroll
-  for (int i = 0; i < 7; ++i) {
-    const float t = mids[i] * s;
-    if (ax > t) idx = i + 1;
-    else if (ax == t && idx == (uint32_t)i) idx = (i & 1) ? i + 1 : i;
-  }
-  return idx == 0 ? 0u : (idx | (x < 0.f ? 8u : 0u));
+// x / s, correctly rounded except within 2^-24 (relative) of a rounding
+// boundary between two floats; exact whenever the quotient is representable.
+__device__ __forceinline__ float quot(float x, float s, float r) {
+  const float q0 = x * r;
+  return fmaf(fmaf(-q0, s, x), r, q0);
+}
+
+// fp32 input only: a quotient on an E2M1 midpoint is moved one ulp toward
+// the side of the exact value (the residual x - q s is exact there).
+__device__ __forceinline__ float off_midpoint(float q, float x, float s) {
+  const float a = fabsf(q);
+  const bool mid = a == 0.25f || a == 0.75f || a == 1.25f || a == 1.75f || a == 2.5f || a == 3.5f || a == 5.0f;
+  if (!mid) return q;
+  const float res = fmaf(-q, s, x);
+  return res > 0.f ? nextafterf(q, INFINITY) : (res < 0.f ? nextafterf(q, -INFINITY) : q);
+}
+
+// Eight E2M1 codes in one word, element k in nibble k (the conversion puts
+// its first operand in the high nibble); magnitude-zero codes lose their sign.
+__device__ __forceinline__ uint32_t e2m1x8(const float* y) {
+  uint32_t w;
+  asm("{ .reg .b8 b0, b1, b2, b3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n"
+      " cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n"
+      " mov.b32 %0, {b0, b1, b2, b3}; }"
+      : "=r"(w)
+      : "f"(y[0]), "f"(y[1]), "f"(y[2]), "f"(y[3]), "f"(y[4]), "f"(y[5]), "f"(y[6]), "f"(y[7]));
+  const uint32_t m = w & 0x77777777u;
+  const uint32_t nz = (m + 0x77777777u) & 0x88888888u;   // bit 3 of a nibble: its magnitude is not 0
+  return w & (0x77777777u | nz);
 }
 
 struct QuantArgs {
@@ -113,8 +147,14 @@ __global__ void __launch_bounds__(256) fp4_quantize_kernel(const QuantArgs a) {
   const float s = e4m3_pos(sb);
   uint32_t w[4] = {0, 0, 0, 0};
   if (s > 0.f) {
+    const float r = 1.0f / s;
 #pragma unroll
-    for (int k = 0; k < 32; ++k) w[k / 8] |= e2m1_code(v[k], s) << (4 * (k % 8));
+    for (int k = 0; k < 32; ++k) {
+      const float q = quot(v[k], s, r);
+      v[k] = BF16 ? q : off_midpoint(q, v[k], s);
+    }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) w[k] = e2m1x8(v + 8 * k);
   }
   *reinterpret_cast<uint4*>(a.codes + dr * a.ld_codes + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
   a.scales[dr * a.ld_scales + b] = (uint8_t)sb;

@@ -57,6 +57,37 @@ def test_fp4_quantize_bitexact():
     assert np.array_equal(_np(codes), codes_ref)
 
 
+def test_fp4_quantize_one_ulp_from_midpoints():
+    """fp32 values one ulp either side of (and exactly on) midpoint x scale,
+    for every E2M1 midpoint, both signs and 59 scales: the quotient x/scale
+    may round onto the midpoint in fp32, and the code must still be the
+    nearest of the exact quotient (ties to even only for exact midpoints)."""
+    mids = np.array([.25, .75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    scales = O.e4m3_decode(np.arange(8, 126, 2))                   # 59 normal E4M3 scales
+    rows = []
+    for sv in scales:
+        # one block per (scale, sign): element 0 = 6 * scale pins the scale to sv exactly
+        for sign in (1.0, -1.0):
+            blk = np.zeros(32, np.float64)
+            blk[0] = 6 * sv
+            k = 1
+            for m in mids:
+                c = np.float32(m * sv)
+                for v in (np.nextafter(c, np.float32(-np.inf)), c, np.nextafter(c, np.float32(np.inf))):
+                    blk[k] = sign * float(v)
+                    k += 1
+            rows.append(blk)
+    x = np.stack(rows).astype(np.float32)                          # [120][32]
+    assert np.all(np.abs(x[:, 0]) == 6 * np.repeat(scales, 2))
+    codes_ref, scales_ref = O.fp4_quantize(x)
+    assert np.array_equal(O.e4m3_decode(scales_ref[:, 0]), np.repeat(scales, 2))
+    codes = torch.zeros((len(x), 16), dtype=torch.uint8, device=DEV)
+    sc = torch.zeros((len(x), 1), dtype=torch.uint8, device=DEV)
+    B.check_status(B.csa2_fp4_quantize(torch.from_numpy(x).to(DEV), codes, sc))
+    assert np.array_equal(_np(sc), scales_ref)
+    assert np.array_equal(_np(codes), codes_ref)
+
+
 def test_fp4_quantize_scatter_rows():
     rng = np.random.default_rng(1)
     x = rng.standard_normal((100, 128)).astype(np.float32)
@@ -432,6 +463,28 @@ def test_plan_verify_block_of_five_queries():
                       modes=(synth.FULL, synth.REINDEX, synth.REUSE))
     c = G.build(wl)
     assert len(c.query_pos) == 5 and (c.seq_of_query == 0).all()
+    _check_plan(c)
+
+
+@pytest.mark.parametrize("case", ["two_reindex_small_heads", "flat_reindex", "paged_one_sequence"])
+def test_plan_one_query_reindex_layers(case):
+    """One query with more candidates than one select CTA holds (the
+    co-resident select) and one or two reindex layers on its pool (the fused
+    reindex launch).  Small heads (4 x d64: 16-column MMA, 64-byte rows) with
+    two reindex layers; all-zero reindex keys, where every pool entry ties and
+    the radix passes decide; 64-row pages."""
+    if case == "two_reindex_small_heads":
+        wl = synth.scaled(synth.C0_TINY, seq_lens=(40000,), pool=2000, topk=64,
+                          modes=(synth.FULL, synth.REINDEX, synth.REINDEX, synth.REUSE))
+    elif case == "flat_reindex":
+        wl = synth.scaled(synth.C1_SINGLE, seq_lens=(40000,), modes=(synth.FULL, synth.REINDEX, synth.REUSE))
+    else:
+        wl = synth.scaled(synth.C3_RAGGED, ragged=(1, 40000, 40000), modes=(synth.FULL, synth.REINDEX))
+    c = G.build(wl)
+    assert len(c.query_pos) == 1 and c.max_ctx > 16384
+    if case == "flat_reindex":
+        c.layers_dev[1].keys.data.zero_()
+        c.host_keys[(1, 0)][:] = 0
     _check_plan(c)
 
 

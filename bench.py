@@ -696,6 +696,9 @@ def run_prefill(args, rank, world, local):
     dev = torch.device(f"cuda:{local}")
     torch.cuda.set_device(dev)
     wl = WL_PREFILL
+    if args.prefill_queries != wl.prefill[0]:   # the last N queries of the chunk (profiling captures)
+        n_ctx = int(wl.lengths()[0])
+        wl = synth.scaled(wl, prefill=(args.prefill_queries, n_ctx - args.prefill_queries))
     t_setup = time.time()
     sq, qp = wl.query_positions()
     nq = len(qp)
@@ -949,6 +952,8 @@ def main():
     ap.add_argument("--impl", default="csa2", choices=["csa2", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--workload", default="decode", choices=WORKLOAD_NAMES)
+    ap.add_argument("--prefill-queries", type=int, default=WL_PREFILL.prefill[0],
+                    help="prefill workload: the last N queries of the chunk (a smaller case for profiling)")
     ap.add_argument("--replicas", type=int, default=0,
                     help="device copies of the state rotated between steps (default: enough to exceed 2x L2)")
     args = ap.parse_args()

@@ -97,7 +97,11 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   int32_t* prefix = w_s + (NG > 128 ? NG : 128);                 // [groups + 1] tiles before each group
   int32_t* gq = prefix + ((a.nq + 2) & ~1);                      // [groups + 1] first query of each group
   int32_t* gseq = gq + ((a.nq + 2) & ~1);                        // [groups] sequence of each group
-  uint64_t* bars = reinterpret_cast<uint64_t*>(gseq + ((a.nq + 2) & ~1));
+  // bit g: the second 64-row box of group g's last tile is visible (its last
+  // position mod 128 is at least 64); with the tile count this is all the
+  // producer needs to know of the positions
+  uint32_t* ghalf = reinterpret_cast<uint32_t*>(gseq + ((a.nq + 2) & ~1));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ghalf + ((a.nq + 63) / 64) * 2);
   uint64_t* full = bars;
   uint64_t* empty = bars + NST;
   uint64_t* tfull = bars + 2 * NST;
@@ -114,7 +118,8 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   const int lane = tid & 31;
   // trace points: 1 prologue done, 2 first TMA issued, 3 first stage landed,
   // 4 first epilogue tile done, 5 last epilogue tile done, 6 histogram
-  // flushed, 7 producer done, 8 MMA issuer done, 9 exit
+  // flushed, 7 producer done, 8 MMA issuer done, 9 exit, 10 producer at its
+  // first ring slot (segment set up)
   CSA2_TRACE_BEGIN(kTrIndex, tid == 0);
   if (tid == 0) prefetch_tensormap(&kmap);   // the descriptor's fetch overlaps the prologue
 
@@ -184,15 +189,18 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     }
     for (int base = 0; base < n_groups; base += 32) {
       const int g = base + lane;
-      int32_t v = 0;
+      int32_t v = 0, last = -1;   // tiles and last visible position of the group
       if (g < n_groups) {
         gseq[g] = a.seq_of_query ? __ldg(a.seq_of_query + gq[g]) : gq[g];   // in flight with the positions
         for (int i = gq[g]; i < gq[g + 1]; ++i) {
           const int32_t pos = __ldg(a.query_pos + i);
           if (pos < 0 || pos >= a.max_ctx) record_error(a.status, CSA2_ERR_INDEX_RANGE);
-          else if ((pos + 128) / 128 > v) v = (pos + 128) / 128;
+          else if (pos > last) last = pos;
         }
+        v = (last + 128) / 128;
       }
+      const uint32_t half = __ballot_sync(0xffffffffu, last >= 0 && (last & 127) >= 64);
+      if (lane == 0) ghalf[base >> 5] = half;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int32_t n = __shfl_up_sync(0xffffffffu, v, o);
@@ -245,11 +253,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
     const int n_it = (int)(s_hi - s_lo);
     const int32_t tile0 = (int32_t)(s_lo - prefix[g]);
     const int q0 = gq[g], nm = gq[g + 1] - gq[g];   // the group's queries
-    int32_t pos_hi = -1;                            // last position any of them sees
-    for (int k = 0; k < nm; ++k) {
-      const int32_t p = __ldg(a.query_pos + q0 + k);
-      if (p < a.max_ctx && p > pos_hi) pos_hi = p;
-    }
+    // box j of tile t is visible unless it is the second box of the group's
+    // last tile and that tile's visible rows end before it
+    const int32_t t_last = prefix[g + 1] - prefix[g] - 1;
+    const bool half = (ghalf[g >> 5] >> (g & 31)) & 1u;
 
     // ---- segment set-up (epilogue threads): B operand = the group's q rows
     // (query k at rows k N .. k N + H - 1, zero rows elsewhere), K-major with
@@ -296,13 +303,14 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       // Lane 0 issues the loads.  With a paged view the whole warp reads the
       // page-table entries one chunk of 16 tiles ahead (lane l: box l & 1 of
       // tile l >> 1 of the chunk), so no load waits on a table lookup.
+      CSA2_MARK(kTrIndex, 10, tid == 0 && git == 0);
       const uint64_t pol = l2_policy_evict_first();
       const int32_t seq = gseq[g];
       const RowMap& m = a.rows;
       auto page_entry = [&](int i0) -> int32_t {   // raw entry behind this lane's box of the chunk at i0
         const int i = i0 + (lane >> 1);
         const int32_t p0 = (tile0 + i) * 128 + 64 * (lane & 1);
-        if (i >= n_it || p0 > pos_hi) return -1;
+        if (i >= n_it || ((lane & 1) && tile0 + i == t_last && !half)) return -1;
         const int32_t pg = p0 / m.page_rows;
         return pg < m.max_pages ? __ldg(m.page_table + (int64_t)seq * m.max_pages + pg) : -1;
       };
@@ -329,7 +337,7 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           } else {
             r[j] = map_row(m, seq, p0);
           }
-          if (p0 > pos_hi) r[j] = -2;   // past the last visible position: no box
+          if (j == 1 && tile == t_last && !half) r[j] = -2;   // past the last visible position: no box
         }
         bool ok = true;
         if (lane == 0) {
@@ -408,6 +416,19 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
 #pragma unroll
         for (int h = 0; h < N; ++h) wreg[h] = w_s[h];
       }
+      // Queries sharing tiles: the head weights of this warp group's query,
+      // four int8 per register for the whole segment (re-reading them from
+      // shared memory for every tile kept the load pipe the busiest unit).
+      constexpr bool kPackW = QG != 1;
+      uint32_t wpk[kPackW ? N / 4 : 1];
+      if constexpr (kPackW) {
+#pragma unroll
+        for (int h4 = 0; h4 < N / 4; ++h4) {
+          const int4 v = *reinterpret_cast<const int4*>(w_s + group * N + 4 * h4);
+          wpk[h4] = (uint32_t)(v.x & 0xFF) | ((uint32_t)(v.y & 0xFF) << 8) | ((uint32_t)(v.z & 0xFF) << 16) |
+                    ((uint32_t)v.w << 24);
+        }
+      }
       for (int i = QG == 1 ? group : 0; i < n_it; i += QG == 1 ? 2 : 1) {
         const int64_t gi = git + i;
         const bool ok = __all_sync(0xffffffffu, mbar_wait(&tfull[gi % NBUF], (uint32_t)((gi / NBUF) & 1), abort_flag));
@@ -440,30 +461,28 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
             }
           }
         } else {
-          // Warp group m reads query m of the tile: its N head dots, 32 (or N)
-          // columns at a time, and the head weights 8 at a time; every warp
-          // frees the buffer once, after its last TMEM read.
-          constexpr int CH = N < 32 ? N : 32;
+          // Warp group m reads query m of the tile: its N head dots 16 columns
+          // at a time (with four partial sums this leaves room for the packed
+          // weights in the 96 registers of an 18-warp CTA); every warp frees
+          // the buffer once, after its last TMEM read.
+          constexpr int CH = 16;
           const int k = group;
           int32_t sc = 0;
           if (ok && k < nm) {
-            int32_t part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            int32_t part[4] = {0, 0, 0, 0};
 #pragma unroll
             for (int c = 0; c < N / CH; ++c) {
               uint32_t rb[CH];
-              if constexpr (CH == 16) tmem_ld16(tbase + (uint32_t)(k * N + c * CH), rb);
-              else tmem_ld32(tbase + (uint32_t)(k * N + c * CH), rb);
+              tmem_ld16(tbase + (uint32_t)(k * N + c * CH), rb);
               tmem_wait_ld();
 #pragma unroll
-              for (int h8 = 0; h8 < CH; h8 += 8) {
-                const int4 w0 = *reinterpret_cast<const int4*>(w_s + k * N + c * CH + h8);
-                const int4 w1 = *reinterpret_cast<const int4*>(w_s + k * N + c * CH + h8 + 4);
-                const int32_t wp[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-#pragma unroll
-                for (int j = 0; j < 8; ++j) part[j] += wp[j] * max((int32_t)rb[h8 + j], 0);
+              for (int j = 0; j < CH; ++j) {
+                const int h = c * CH + j;
+                const int32_t wv = (int32_t)(int8_t)(wpk[h >> 2] >> (8 * (h & 3)));
+                part[j & 3] += wv * max((int32_t)rb[j], 0);
               }
             }
-            sc = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+            sc = (part[0] + part[1]) + (part[2] + part[3]);
           }
           tc_fence_before();
           __syncwarp();
@@ -547,7 +566,7 @@ size_t index_smem_bytes(int N, int QG, int nq) {
   using Cfg = IndexCfg<D>;
   const int NG = N * QG;
   return 1024 + (size_t)Cfg::kStages * Cfg::kTile + (size_t)NG * D + (QG == 1 ? kBuckets * 4 : 0) +
-         (size_t)(NG > 128 ? NG : 128) * 4 + 3 * (size_t)((nq + 2) & ~1) * 4 + (2 * Cfg::kStages + 2 * 8) * 8 +
+         (size_t)(NG > 128 ? NG : 128) * 4 + 3 * (size_t)((nq + 2) & ~1) * 4 + (size_t)((nq + 63) / 64) * 8 + (2 * Cfg::kStages + 2 * 8) * 8 +
          32 + 8 * (size_t)QG + 4 * (size_t)QG + 16;
 }
 

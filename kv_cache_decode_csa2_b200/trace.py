@@ -32,7 +32,7 @@ POINTS = 16
 POINT_NAMES = {
     0: ("index_score", ["entry", "prologue done", "first TMA issued", "first stage landed",
                         "first epilogue tile", "last epilogue tile", "histogram flushed", "producer done",
-                        "MMA issuer done", "exit"]),
+                        "MMA issuer done", "exit", "producer set up"]),
     1: ("select", ["entry", "grid before done", "threshold buckets", "classified", "first grid barrier",
                    "row ties staged", "ties ranked", "second grid barrier", "written"]),
     2: ("reindex_select", ["entry", "own inputs staged", "grid before done", "pool rows gathered", "scored",

@@ -572,8 +572,10 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
   const dim3 grid(s.n_chunks, nq);
   cudaError_t e;
   // Many rows that do not fit on the device at once: one CTA per row, which
-  // builds its own histogram.
-  if (!select_fits(nq, n_max) && n_max <= kRowSelMax)
+  // builds its own histogram.  Fewer rows than half the SMs (a decode batch of
+  // long sequences) would leave most SMs idle that way: they take the chunked
+  // passes below, which spread every row over many CTAs.
+  if (!select_fits(nq, n_max) && n_max <= kRowSelMax && 2 * nq >= sm_count())
     return launch_row_select(scores, ld, n_valid, query_pos, cand_pos, nq, n_max, outs, n_k, status, st);
   if (!hist_ready) {
     e = cudaMemsetAsync(s.hist, 0, topk_zero_bytes(nq), st);

@@ -180,8 +180,9 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
       if (lane == 0) gq[n_groups] = a.nq;
       __syncwarp();
     }
-    // prefix[g+1] = tiles up to group g: a group's tiles cover the longest
-    // causal prefix of its queries
+    // prefix[g+1] = work units up to group g (a group's tiles cover the
+    // longest causal prefix of its queries; one unit per tile, or 3 + its
+    // queries per tile in a grouped launch)
     int32_t carry = 0;
     if (lane == 0) {
       prefix[0] = 0;
@@ -198,6 +199,10 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
           else if (pos > last) last = pos;
         }
         v = (last + 128) / 128;
+        // grouped launches divide work units, not tiles, among the CTAs: a
+        // tile costs about 3 + (its group's queries) units (the epilogue's
+        // share grows with the queries, the stream's does not)
+        if constexpr (QG != 1) v *= 3 + (gq[g + 1] - gq[g]);
       }
       const uint32_t half = __ballot_sync(0xffffffffu, last >= 0 && (last & 127) >= 64);
       if (lane == 0) ghalf[base >> 5] = half;
@@ -250,12 +255,18 @@ index_score_kernel(const __grid_constant__ CUtensorMap kmap, const IndexArgs a) 
   for (int64_t s_lo = lo; s_lo < hi;) {
     while (s_lo >= prefix[g + 1]) ++g;
     const int64_t s_hi = hi < (int64_t)prefix[g + 1] ? hi : (int64_t)prefix[g + 1];
-    const int n_it = (int)(s_hi - s_lo);
-    const int32_t tile0 = (int32_t)(s_lo - prefix[g]);
     const int q0 = gq[g], nm = gq[g + 1] - gq[g];   // the group's queries
+    // the tiles of group g whose first work unit lies in [s_lo, s_hi)
+    const int32_t wu = QG == 1 ? 1 : 3 + nm;
+    const int32_t tile0 = (int32_t)((s_lo - prefix[g] + wu - 1) / wu);
+    const int n_it = (int)((s_hi - prefix[g] + wu - 1) / wu) - tile0;
+    if (n_it <= 0) {   // (every thread agrees) no tile starts in this range
+      s_lo = s_hi;
+      continue;
+    }
     // box j of tile t is visible unless it is the second box of the group's
     // last tile and that tile's visible rows end before it
-    const int32_t t_last = prefix[g + 1] - prefix[g] - 1;
+    const int32_t t_last = (prefix[g + 1] - prefix[g]) / wu - 1;
     const bool half = (ghalf[g >> 5] >> (g & 31)) & 1u;
 
     // ---- segment set-up (epilogue threads): B operand = the group's q rows

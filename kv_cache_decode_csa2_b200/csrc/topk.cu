@@ -277,6 +277,8 @@ __device__ uint64_t radix_select(Get get, int64_t m, int64_t need, uint32_t* his
 
 // ------------------------------------------------------------------ hist
 __global__ void __launch_bounds__(256) topk_hist_kernel(CandView v, uint32_t* hist) {
+  pdl_wait();      // the scores come from the grid before
+  pdl_trigger();
   __shared__ uint32_t h[kBuckets];
   const int q = blockIdx.y;
   const int32_t n = n_of(v, q);
@@ -298,8 +300,12 @@ __global__ void __launch_bounds__(256) topk_hist_kernel(CandView v, uint32_t* hi
     if (j < n) atomicAdd(&h[score_bucket(sr[i])], 1u);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x)
-    if (h[i]) atomicAdd(hist + (int64_t)q * kBuckets + i, h[i]);
+  // one 64-bit add per populated pair of buckets (no carry: a count stays below 2^32)
+  unsigned long long* gh = reinterpret_cast<unsigned long long*>(hist + (int64_t)q * kBuckets);
+  for (int i = threadIdx.x; i < kBuckets / 2; i += blockDim.x) {
+    const uint32_t lo = h[2 * i], hi = h[2 * i + 1];
+    if (lo | hi) atomicAdd(gh + i, (unsigned long long)lo | ((unsigned long long)hi << 32));
+  }
 }
 
 // ------------------------------------------------------------------ thresholds
@@ -314,6 +320,12 @@ __global__ void __launch_bounds__(256) topk_thresh_kernel(ThreshArgs a) {
   __shared__ int32_t tmp[32];
   __shared__ int32_t b_s, above_s;
   const int q = blockIdx.x;
+  pdl_wait();      // the histogram comes from the grids before
+  pdl_trigger();
+  // the gather's published chunk counts start at zero (the gather runs after
+  // this grid has completed)
+  unsigned long long* pub = reinterpret_cast<unsigned long long*>(a.s.chunk_cnt) + (int64_t)q * 2 * a.s.n_chunks;
+  for (int i = threadIdx.x; i < 2 * a.s.n_chunks; i += blockDim.x) pub[i] = 0ull;
   const uint32_t* hist = a.s.hist + (int64_t)q * kBuckets;
   for (int t = 0; t < a.n_k; ++t) {
     find_threshold<256>(hist, a.k[t], &b_s, &above_s, tmp);
@@ -342,6 +354,8 @@ __device__ __forceinline__ unsigned long long ld_relaxed_u64(const unsigned long
 }
 
 __global__ void __launch_bounds__(256) topk_gather_kernel(GatherArgs a) {
+  pdl_wait();      // scores, thresholds and zeroed counts come from the grids before
+  pdl_trigger();
   __shared__ int32_t tmp[32];
   __shared__ int32_t base_s;
   const int q = blockIdx.y, c = blockIdx.x;
@@ -436,6 +450,8 @@ constexpr int kFinishPer = (kCandCap + 1023) / 1024;   // list keys per thread: 
 // over shared memory.  The ordered write uses per-(pass, warp) member counts,
 // as in the one-CTA kernel.
 __global__ void __launch_bounds__(1024, 1) topk_finish_kernel(FinishArgs a) {
+  pdl_wait();      // the candidate lists come from the grid before
+  pdl_trigger();
   extern __shared__ uint64_t keys_s[];            // [cand_cap] then [kTieCap] ties
   uint64_t* ties = keys_s + kCandCap;
   __shared__ int32_t cmat[kFinishPer * 32];
@@ -577,28 +593,31 @@ cudaError_t launch_topk_large(const int32_t* scores, int64_t ld, const int32_t* 
   // passes below, which spread every row over many CTAs.
   if (!select_fits(nq, n_max) && n_max <= kRowSelMax && 2 * nq >= sm_count())
     return launch_row_select(scores, ld, n_valid, query_pos, cand_pos, nq, n_max, outs, n_k, status, st);
+  const bool pdl = launch_opts().pdl;
   if (!hist_ready) {
     e = cudaMemsetAsync(s.hist, 0, topk_zero_bytes(nq), st);
     if (e != cudaSuccess) return e;
-    topk_hist_kernel<<<grid, 256, 0, st>>>(v, s.hist);
+    e = launch_k(topk_hist_kernel, grid, dim3(256), 0, st, false, false, v, s.hist);
+    if (e != cudaSuccess) return e;
   }
   // One pass of co-resident select CTAs when the rows fit on the device.
   e = launch_select(scores, ld, n_valid, query_pos, cand_pos, nq, n_max, outs, n_k, s.hist, &s, status, st);
   if (e != cudaErrorNotSupported) return e;
   (void)cudaGetLastError();
-  e = cudaMemsetAsync(s.chunk_cnt, 0, (size_t)nq * 2 * s.n_chunks * 8, st);
-  if (e != cudaSuccess) return e;
+  // thresholds (which also zero the gather's chunk counts), gather, finish:
+  // programmatic dependents of one another within a plan step
   ThreshArgs ta{s, {outs[0].k, n_k > 1 ? outs[1].k : 0}, n_k};
-  topk_thresh_kernel<<<nq, 256, 0, st>>>(ta);
+  e = launch_k(topk_thresh_kernel, dim3(nq), dim3(256), 0, st, false, pdl, ta);
+  if (e != cudaSuccess) return e;
   GatherArgs ga{v, s, n_k, status};
-  topk_gather_kernel<<<grid, 256, 0, st>>>(ga);
+  e = launch_k(topk_gather_kernel, grid, dim3(256), 0, st, false, pdl, ga);
+  if (e != cudaSuccess) return e;
   const int smem = (kCandCap + kTieCap) * 8;
   static SetupMask done{0};
   e = ensure_smem(topk_finish_kernel, smem, done);
   if (e != cudaSuccess) return e;
   FinishArgs fa{v, s, {outs[0], n_k > 1 ? outs[1] : outs[0]}};
-  topk_finish_kernel<<<dim3(nq, n_k), 1024, smem, st>>>(fa);
-  return cudaGetLastError();
+  return launch_k(topk_finish_kernel, dim3(nq, n_k), dim3(1024), smem, st, false, pdl, fa);
 }
 
 cudaError_t launch_topk_small(const int32_t* scores, int64_t ld, const int32_t* n_valid,

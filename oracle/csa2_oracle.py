@@ -45,7 +45,14 @@ see tests/test_oracle_pins.py):
                       ml_dtypes' float -> float4_e2m1fn rounding inside the range.
   sparse_attention    pinned: torch scaled_dot_product_attention (fp64) when
                       the set is the whole context; closed forms.
+  full_index, reindex, attention_set
+                      compositions of the pinned functions above (scores, then
+                      the top-k of all positions or of the pool; the set
+                      selection U window); pinned with the plan's brute force.
   decode_layer_plan   pinned: separate pure-Python brute force on tiny inputs.
+                      Which keys a reindex layer reads and what the full layer
+                      attends to are READINGS 3 and 4 (parity unpinned by the
+                      pages).
   prefill_query       pinned: equals decode at the same position (property).
   attention_combine   pinned: equals sparse_attention over the union on random
                       partitions (one set empty), and the single-set identity.

@@ -248,34 +248,32 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   CSA2_MARK(kTrRowSel, 2, tid == 0);
   const long long lo0 = bound_s[0], hi0 = bound_s[1], lo1 = bound_s[2], hi1 = bound_s[3];
   const bool all0 = b0 < 0, all1 = n_k > 1 && b1 < 0;
+  // Word x of the bitmasks covers candidates j0 + 32 x .. j0 + 32 x + 31.  The
+  // word loop stays rolled (this code runs once per row, from a cold
+  // instruction cache): each word's masks come from branch-free comparisons
+  // and are shifted into the register arrays, so that word x ends at index
+  // kRowWords - 1 - x with every index a constant.
   uint32_t above_m[NK][kRowWords], tie_m[NK][kRowWords];
 #pragma unroll
   for (int t = 0; t < NK; ++t)
 #pragma unroll
     for (int w = 0; w < kRowWords; ++w) above_m[t][w] = tie_m[t][w] = 0u;
-  // word x of the bitmasks covers candidates j0 + 32 x .. j0 + 32 x + 31
-#pragma unroll
+#pragma unroll 1
   for (int x = 0; x < kRowWords; ++x) {
     const int32_t base = j0 + 32 * x;
-    if (base < j1) {
-      auto take = [&](int e, int32_t s) {
-        const uint32_t bit = 1u << e;
-        if (all0 || s >= hi0) above_m[0][x] |= bit;   // b* = -1 takes every candidate
-        if (NK > 1 && (all1 || s >= hi1)) above_m[NK - 1][x] |= bit;
-        const bool t0 = !all0 && s >= lo0 && s < hi0;
-        const bool t1 = NK > 1 && !all1 && s >= lo1 && s < hi1;
-        if (t0 || t1) {
-          const uint64_t key = cand_key(s, base + e);
+    uint32_t am[NK], tm[NK];
 #pragma unroll
-          for (int t = 0; t < NK; ++t) {
-            if (t ? t1 : t0) {
-              tie_m[t][x] |= bit;
-              const uint32_t slot = atomicAdd(&nt_s[t], 1u);
-              if (slot < (uint32_t)kRowTieCap) ties[t * kRowTieCap + slot] = key;
-            }
-          }
-        }
-      };
+    for (int t = 0; t < NK; ++t) am[t] = tm[t] = 0u;
+    auto take = [&](int e, int32_t sv) {
+      const long long s = sv;
+      am[0] |= (uint32_t)(all0 || s >= hi0) << e;   // b* = -1 takes every candidate
+      tm[0] |= (uint32_t)(!all0 && s >= lo0 && s < hi0) << e;
+      if constexpr (NK > 1) {
+        am[NK - 1] |= (uint32_t)(all1 || s >= hi1) << e;
+        tm[NK - 1] |= (uint32_t)(!all1 && s >= lo1 && s < hi1) << e;
+      }
+    };
+    if (base < j1) {
       if (vec && base + 32 <= j1) {
         int4 v[8];
 #pragma unroll
@@ -288,7 +286,33 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
           take(4 * u + 3, v[u].w);
         }
       } else {
+#pragma unroll 1
         for (int e = 0; e < 32 && base + e < j1; ++e) take(e, __ldcg(row + base + e));
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < NK; ++t) {
+#pragma unroll
+      for (int w = kRowWords - 1; w > 0; --w) {
+        above_m[t][w] = above_m[t][w - 1];
+        tie_m[t][w] = tie_m[t][w - 1];
+      }
+      above_m[t][0] = am[t];
+      tie_m[t][0] = tm[t];
+    }
+  }
+  // the ties (few) go to the row's list; their scores are read again
+#pragma unroll
+  for (int t = 0; t < NK; ++t) {
+#pragma unroll
+    for (int x = 0; x < kRowWords; ++x) {
+      uint32_t tmk = tie_m[t][kRowWords - 1 - x];
+      while (tmk) {
+        const int b = __ffs(tmk) - 1;
+        tmk &= tmk - 1u;
+        const int32_t j = j0 + 32 * x + b;
+        const uint32_t slot = atomicAdd(&nt_s[t], 1u);
+        if (slot < (uint32_t)kRowTieCap) ties[t * kRowTieCap + slot] = cand_key(__ldcg(row + j), j);
       }
     }
   }
@@ -374,14 +398,14 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   for (int t = 0; t < NK; ++t) {
 #pragma unroll
     for (int x = 0; x < kRowWords; ++x) {
-      uint32_t tm = tie_m[t][x];
+      uint32_t tm = tie_m[t][kRowWords - 1 - x];
       while (tm) {   // ties are few: read their scores again
         const int b = __ffs(tm) - 1;
         tm &= tm - 1u;
         const int32_t j = j0 + x * 32 + b;
-        if (cand_key(__ldcg(row + j), j) >= kthr[t]) above_m[t][x] |= 1u << b;
+        if (cand_key(__ldcg(row + j), j) >= kthr[t]) above_m[t][kRowWords - 1 - x] |= 1u << b;
       }
-      cnt[t] += __popc(above_m[t][x]);
+      cnt[t] += __popc(above_m[t][kRowWords - 1 - x]);
     }
   }
   uint64_t tot;
@@ -394,7 +418,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     int64_t slot = (int64_t)((ex >> (32 * t)) & 0xffffffffu);
 #pragma unroll
     for (int x = 0; x < kRowWords; ++x) {
-      uint32_t m = above_m[t][x];
+      uint32_t m = above_m[t][kRowWords - 1 - x];
       while (m) {
         const int b = __ffs(m) - 1;
         m &= m - 1u;

@@ -209,6 +209,66 @@ def test_topk_many_long_rows(spread, k):
         assert (o[i, c[i]:] == -1).all()
 
 
+@pytest.mark.parametrize("spread,k,with_pos", [(10 ** 6, 700, False), (1000, 512, True), (2, 600, False),
+                                                (0, 512, True)])
+def test_topk_one_cta_per_row(spread, k, with_pos):
+    """80 rows of up to 50,000 candidates: at least half as many rows as SMs
+    and too long for the co-resident select, so each row takes one CTA of the
+    row kernel (the 40- and 24-row cases above take the chunked passes).
+    Spreads 2 and 0 overflow the tie list; ragged valid counts include one
+    below k and one inside a single select span."""
+    rng = np.random.default_rng(7 * spread + k)
+    nq, n = 80, 50000
+    s = rng.integers(-spread, spread + 1, size=(nq, n)).astype(np.int32)
+    nv = rng.integers(n // 2, n + 1, size=nq).astype(np.int32)
+    nv[5], nv[6], nv[7] = k // 2, 9000, n
+    pos = None
+    if with_pos:
+        pos = np.sort(rng.choice(10 ** 7, size=(nq, n), replace=True), axis=1).astype(np.int32)
+        pos += np.arange(n, dtype=np.int32)[None]
+    out = torch.empty((nq, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((nq,), dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_topk_pool(torch.from_numpy(s).to(DEV), k, out, out_cnt=cnt,
+                                    n_valid=torch.from_numpy(nv).to(DEV),
+                                    cand_pos=None if pos is None else torch.from_numpy(pos).to(DEV)))
+    o, c = _np(out), _np(cnt)
+    for i in range(nq):
+        p_i = np.arange(nv[i]) if pos is None else pos[i, :nv[i]]
+        ref = O.top_k_positions(s[i, :nv[i]], p_i, k)
+        assert c[i] == len(ref) and np.array_equal(o[i, :c[i]], ref), f"row {i}"
+        assert (o[i, c[i]:] == -1).all()
+
+
+@pytest.mark.parametrize("mode", ["random", "half"])
+def test_index_full_prefill_pool_and_selection_rows(mode):
+    """80 causal queries at the end of a 50,000-row sequence, each keeping a
+    pool of 16,384 and a top-512: the row kernel with both targets in one
+    pass.  Half-zero keys put thousands of equal zero scores at the pool's
+    threshold.  Sampled queries are checked against the oracle one by one."""
+    ctx, nq, P, K = 50000, 80, 16384, 512
+    wl = synth.scaled(synth.C1_SINGLE, seq_lens=(ctx,), prefill=(nq, ctx - nq), pool=P, topk=K)
+    c = G.build(wl, fp4_on_gpu=True)   # only the index side is checked here
+    ly = c.layers_dev[0]
+    keys = c.host_keys[(0, 0)].copy()
+    if mode == "half":
+        keys[::2] = 0
+        ly.keys.data[:ctx].copy_(torch.from_numpy(keys))
+    pool = torch.full((nq, P), -7, dtype=torch.int32, device=DEV)
+    pcnt = torch.full((nq,), -7, dtype=torch.int32, device=DEV)
+    sel = torch.full((nq, K), -7, dtype=torch.int32, device=DEV)
+    scnt = torch.full((nq,), -7, dtype=torch.int32, device=DEV)
+    B.check_status(B.csa2_index_full(ly.q, ly.w, ly.keys, c.pos_dev, c.max_ctx, seq_of_query=c.seq_dev,
+                                     P=P, pool_idx=pool, pool_cnt=pcnt, K=K, sel_idx=sel, sel_cnt=scnt))
+    po, pc, so, sc = _np(pool), _np(pcnt), _np(sel), _np(scnt)
+    for i in (0, 1, 40, 78, 79):
+        q, w = c.host_q[(0, i)]
+        _, ref_pool, ref_sel = O.full_index(q, w, keys, int(c.query_pos[i]), P, K)
+        assert pc[i] == len(ref_pool) and np.array_equal(po[i, :pc[i]], ref_pool), f"query {i} pool"
+        assert (po[i, pc[i]:] == -1).all()
+        assert sc[i] == len(ref_sel) and np.array_equal(so[i, :sc[i]], ref_sel), f"query {i} selection"
+        assert (so[i, sc[i]:] == -1).all()
+
+
 def test_topk_many_long_rows_with_positions():
     rng = np.random.default_rng(9)
     nq, n = 24, 70000

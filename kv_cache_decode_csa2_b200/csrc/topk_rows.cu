@@ -8,16 +8,23 @@
 //   pass 1  bucket histogram of the row in shared memory, counting only
 //           candidates at or above a cut that a small sample of the row
 //           picks (with a full-histogram redo should too few clear it); one
-//           block scan finds the threshold bucket b* of each target;
-//   pass 2  per-thread bitmasks of the members above b* and of the ties at
-//           b*; the ties go to a shared list, each warp ranks some of them
+//           block scan finds the threshold bucket b* of each target.  Each
+//           thread also keeps its first kRowKeep candidates at or above the
+//           cut (score and offset) in shared memory;
+//   pass 2  when no thread kept more than kRowKeep, every member is among
+//           the kept candidates (b* is at or above the cut), and the ties at
+//           b* come from them; otherwise the row is read again into
+//           per-thread bitmasks of the members above b* and of the ties.
+//           The ties go to a shared list, each warp ranks some of them
 //           against it, and this gives the smallest member tie key;
 //   write   one packed block scan of the member counts gives every thread
 //           its first output slot; the members are written in position
-//           order from the bitmasks, without reading the scores again.
-// A row reads its scores twice.  A tie list longer than kRowTieCap (a very
-// flat score distribution) is resolved by a radix select of the k-th tie key,
-// one 8-bit digit per pass over the row.
+//           order from the kept list or the bitmasks.
+// A row reads its scores once when the cut is selective (about 2.5
+// candidates per thread clear it for a top-512 of 262,144), else twice.  A
+// tie list longer than kRowTieCap (a very flat score distribution) is
+// resolved by a radix select of the k-th tie key, one 8-bit digit per pass
+// over the row.
 #include "csa2_device.cuh"
 #include "internal.h"
 #include "select_common.cuh"
@@ -31,7 +38,9 @@ namespace {
 constexpr int kRowNT = 1024;
 constexpr int kRowWords = kRowPer / 32;   // bitmask words per thread and target
 constexpr int kRowTieCap = 4096;
+constexpr int kRowKeep = 16;               // kept candidates per thread
 static_assert(kRowPer % 32 == 0 && kBuckets / kRowNT == 8, "shapes");
+static_assert(kRowPer <= 256, "a kept candidate's offset is one byte");
 
 struct RowArgs {
   const int32_t* scores;
@@ -64,6 +73,8 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   extern __shared__ __align__(16) unsigned char row_dyn[];
   uint32_t* hist = reinterpret_cast<uint32_t*>(row_dyn);                      // [kBuckets]
   uint64_t* ties = reinterpret_cast<uint64_t*>(row_dyn + kBuckets * 4);       // [2][kRowTieCap]
+  int32_t* keep_s = reinterpret_cast<int32_t*>(ties + 2 * kRowTieCap);        // [kRowKeep][kRowNT]
+  uint8_t* keep_o = reinterpret_cast<uint8_t*>(keep_s + kRowKeep * kRowNT);   // [kRowKeep][kRowNT]
   __shared__ uint64_t wtmp[32];
   __shared__ int32_t bstar_s[2], above_s[2];
   __shared__ uint32_t nt_s[2];
@@ -166,9 +177,25 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   if (tid == 0) cut_score_s = bucket_min_score(cut_s);
   __syncthreads();
   const int32_t cut_score = cut_score_s;
+  // candidates of this thread at or above the cut; the first kRowKeep are kept
+  int32_t n_kept = 0;
+  bool kept_all = true;   // the kept list holds every candidate at or above the cut
 #pragma unroll 1
   for (int attempt = 0; attempt < 2; ++attempt) {
     const int32_t lo_s = attempt == 0 ? cut_score : INT32_MIN;   // count scores >= lo_s
+    const bool keep = attempt == 0;
+    auto count = [&](int32_t off, int32_t sv) {
+      if (sv >= lo_s) {   // about one candidate in a hundred above a sampled cut
+        atomicAdd(&hist[score_bucket(sv)], 1u);
+        if (keep) {
+          if (n_kept < kRowKeep) {
+            keep_s[n_kept * kRowNT + tid] = sv;
+            keep_o[n_kept * kRowNT + tid] = (uint8_t)off;
+          }
+          ++n_kept;
+        }
+      }
+    };
     // words of 32 candidates; a word's eight loads are all issued before any is used
 #pragma unroll 1
     for (int x = 0; x < kRowWords; ++x) {
@@ -180,18 +207,17 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
         for (int u = 0; u < 8; ++u) v[u] = __ldcg(reinterpret_cast<const int4*>(row + base) + u);
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int32_t sv[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            if (sv[e] >= lo_s) atomicAdd(&hist[score_bucket(sv[e])], 1u);
+          count(32 * x + 4 * u, v[u].x);
+          count(32 * x + 4 * u + 1, v[u].y);
+          count(32 * x + 4 * u + 2, v[u].z);
+          count(32 * x + 4 * u + 3, v[u].w);
         }
       } else {
-        for (int e = 0; e < 32 && base + e < j1; ++e) {
-          const int32_t sv = __ldcg(row + base + e);
-          if (sv >= lo_s) atomicAdd(&hist[score_bucket(sv)], 1u);
-        }
+#pragma unroll 1
+        for (int e = 0; e < 32 && base + e < j1; ++e) count(32 * x + e, __ldcg(row + base + e));
       }
     }
+    if (attempt == 1) kept_all = false;   // the redo counted below the cut: the list is partial
     if (attempt == 0 && a.cand_pos) {   // candidate positions must ascend
       const int32_t* cp = a.cand_pos + (int64_t)q * a.ld;
       bool bad = false;
@@ -230,10 +256,11 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     }
     __syncthreads();
   }
-  __syncthreads();
+  // every member is kept when every thread kept all it counted above the cut
+  const bool fast = __syncthreads_and(kept_all && n_kept <= kRowKeep) != 0;
   CSA2_MARK(kTrRowSel, 1, tid == 0);
 
-  // ---- pass 2: members above b* and ties at b*, as bitmasks
+  // ---- pass 2: members above b* and ties at b*, from the kept list or as bitmasks
   const int32_t b0 = bstar_s[0], b1 = n_k > 1 ? bstar_s[1] : INT32_MIN;
   // score ranges: above b* means s >= hi_t, at b* means lo_t <= s < hi_t
   // (64-bit: the bucket above the top one starts past every int32 score)
@@ -258,8 +285,23 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   for (int t = 0; t < NK; ++t)
 #pragma unroll
     for (int w = 0; w < kRowWords; ++w) above_m[t][w] = tie_m[t][w] = 0u;
+  auto add_tie = [&](int t, int32_t sv, int32_t j) {
+    const uint32_t slot = atomicAdd(&nt_s[t], 1u);
+    if (slot < (uint32_t)kRowTieCap) ties[t * kRowTieCap + slot] = cand_key(sv, j);
+  };
+  if (fast) {   // the kept candidates: offsets ascend with the slot
 #pragma unroll 1
-  for (int x = 0; x < kRowWords; ++x) {
+    for (int c = 0; c < n_kept; ++c) {
+      const int32_t sv = keep_s[c * kRowNT + tid];
+      const int32_t j = j0 + keep_o[c * kRowNT + tid];
+      const long long sl = sv;
+      if (!all0 && sl >= lo0 && sl < hi0) add_tie(0, sv, j);
+      if constexpr (NK > 1)
+        if (!all1 && sl >= lo1 && sl < hi1) add_tie(1, sv, j);
+    }
+  }
+#pragma unroll 1
+  for (int x = 0; x < (fast ? 0 : kRowWords); ++x) {
     const int32_t base = j0 + 32 * x;
     uint32_t am[NK], tm[NK];
 #pragma unroll
@@ -302,6 +344,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     }
   }
   // the ties (few) go to the row's list; their scores are read again
+  // (the masks are all zero on the kept-list path)
 #pragma unroll
   for (int t = 0; t < NK; ++t) {
 #pragma unroll
@@ -311,8 +354,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
         const int b = __ffs(tmk) - 1;
         tmk &= tmk - 1u;
         const int32_t j = j0 + 32 * x + b;
-        const uint32_t slot = atomicAdd(&nt_s[t], 1u);
-        if (slot < (uint32_t)kRowTieCap) ties[t * kRowTieCap + slot] = cand_key(__ldcg(row + j), j);
+        add_tie(t, __ldcg(row + j), j);
       }
     }
   }
@@ -394,6 +436,22 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   // ---- members: ties at or above the threshold key join the bitmasks
   const uint64_t kthr[2] = {kthr_s[0], kthr_s[1]};
   uint32_t cnt[2] = {0u, 0u};
+  // kept-list path: a member is above b*, or a tie whose key is at least the
+  // threshold key (a target that takes every candidate kept them all)
+  auto member = [&](int t, int32_t sv, int32_t j) -> bool {
+    const long long sl = sv;
+    if (t == 0) return all0 || sl >= hi0 || (sl >= lo0 && cand_key(sv, j) >= kthr[0]);
+    return all1 || sl >= hi1 || (sl >= lo1 && cand_key(sv, j) >= kthr[1]);
+  };
+  if (fast) {
+#pragma unroll 1
+    for (int c = 0; c < n_kept; ++c) {
+      const int32_t sv = keep_s[c * kRowNT + tid];
+      const int32_t j = j0 + keep_o[c * kRowNT + tid];
+#pragma unroll
+      for (int t = 0; t < NK; ++t) cnt[t] += member(t, sv, j) ? 1u : 0u;
+    }
+  }
 #pragma unroll
   for (int t = 0; t < NK; ++t) {
 #pragma unroll
@@ -416,6 +474,17 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
     const int32_t k = a.k[t];
     int32_t* dst = a.out_idx[t] + (int64_t)q * k;
     int64_t slot = (int64_t)((ex >> (32 * t)) & 0xffffffffu);
+    if (fast) {
+#pragma unroll 1
+      for (int c = 0; c < n_kept; ++c) {
+        const int32_t sv = keep_s[c * kRowNT + tid];
+        const int32_t j = j0 + keep_o[c * kRowNT + tid];
+        if (member(t, sv, j)) {
+          if (slot < k) dst[slot] = cp ? __ldg(cp + j) : j;
+          ++slot;
+        }
+      }
+    }
 #pragma unroll
     for (int x = 0; x < kRowWords; ++x) {
       uint32_t m = above_m[t][kRowWords - 1 - x];
@@ -435,7 +504,7 @@ __global__ void __launch_bounds__(kRowNT, 1) row_select_kernel(const __grid_cons
   CSA2_MARK(kTrRowSel, 5, tid == 0);
 }
 
-constexpr int kRowSmem = kBuckets * 4 + 2 * kRowTieCap * 8;
+constexpr int kRowSmem = kBuckets * 4 + 2 * kRowTieCap * 8 + kRowKeep * kRowNT * 5;
 
 }  // namespace
 

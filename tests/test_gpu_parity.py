@@ -215,8 +215,10 @@ def test_topk_one_cta_per_row(spread, k, with_pos):
     """80 rows of up to 50,000 candidates: at least half as many rows as SMs
     and too long for the co-resident select, so each row takes one CTA of the
     row kernel (the 40- and 24-row cases above take the chunked passes).
-    Spreads 2 and 0 overflow the tie list; ragged valid counts include one
-    below k and one inside a single select span."""
+    Wide spreads keep the few candidates above the sampled cut in shared
+    memory; spreads 2 and 0 put too many there (the row is read again) and
+    overflow the tie list; ragged valid counts include one below k and one
+    inside a single select span."""
     rng = np.random.default_rng(7 * spread + k)
     nq, n = 80, 50000
     s = rng.integers(-spread, spread + 1, size=(nq, n)).astype(np.int32)
@@ -239,13 +241,15 @@ def test_topk_one_cta_per_row(spread, k, with_pos):
         assert (o[i, c[i]:] == -1).all()
 
 
-@pytest.mark.parametrize("mode", ["random", "half"])
-def test_index_full_prefill_pool_and_selection_rows(mode):
+@pytest.mark.parametrize("mode,P,K", [("random", 16384, 512), ("half", 16384, 512), ("random", 1024, 256)])
+def test_index_full_prefill_pool_and_selection_rows(mode, P, K):
     """80 causal queries at the end of a 50,000-row sequence, each keeping a
-    pool of 16,384 and a top-512: the row kernel with both targets in one
-    pass.  Half-zero keys put thousands of equal zero scores at the pool's
+    pool and a top-K: the row kernel with both targets in one pass.  A pool
+    of 16,384 makes its sampled cut loose (the row is read twice); a pool of
+    1,024 keeps the candidates above the cut in shared memory (read once).
+    Half-zero keys put thousands of equal zero scores at the pool's
     threshold.  Sampled queries are checked against the oracle one by one."""
-    ctx, nq, P, K = 50000, 80, 16384, 512
+    ctx, nq = 50000, 80
     wl = synth.scaled(synth.C1_SINGLE, seq_lens=(ctx,), prefill=(nq, ctx - nq), pool=P, topk=K)
     c = G.build(wl, fp4_on_gpu=True)   # only the index side is checked here
     ly = c.layers_dev[0]

@@ -14,6 +14,9 @@ Workloads (--workload):
             table), one full layer each: queries/s.
   verify    a speculative-verify block of 5 causal queries at the end of the
             1M context, all 8 layers, the index scan shared by the block.
+  window    the decode step with a local window cache per layer: every layer
+            reads its 128-token window from its own bf16 ring, every reuse
+            layer reads the FP4 cache of the layer whose selection it reuses.
   prefill   2048 causal queries at positions 260096-262143 of a 262,144-row
             context: int8 index GEMM, per-query top-512 over the prefix,
             attention.  queries/s and the index stage's int8 TOP/s.
@@ -67,6 +70,10 @@ METRIC = "decode steps/s and HBM GB/s (% of B200 roofline) at 1M-token context"
 WL = synth.C2_1M_PLAN
 WL_VERIFY = synth.scaled(synth.C2_1M_PLAN, name="verify_5q_ctx1048576_8layer",
                          prefill=(5, int(synth.C2_1M_PLAN.lengths()[0]) - 5))
+WL_WINDOW = synth.scaled(synth.C2_1M_PLAN, name="window_ctx1048576_8layer")
+# workloads whose layers read their window from a local bf16 ring and whose
+# reuse layers share the global FP4 cache of the layer they reuse
+LOCAL_WINDOW_WORKLOADS = ("window",)
 # name: (workload, metric, unit, units per step, group the queries of a sequence)
 DECODE_WORKLOADS = {
     "decode": (WL, METRIC, "steps/s", 1, False),
@@ -77,6 +84,8 @@ DECODE_WORKLOADS = {
                "queries/s", 32, False),
     "verify": (WL_VERIFY, "verify blocks/s (5 queries sharing one index scan) at 1M-token context",
                "blocks/s", 1, True),
+    "window": (WL_WINDOW, "decode steps/s at 1M-token context with per-layer local window caches (bf16) and "
+                          "reuse layers sharing the global FP4 KV", "steps/s", 1, False),
 }
 METRIC_PREFILL = "prefill-chunk queries/s and index int8 TOP/s (2048 causal queries, 262144 context)"
 WL_PREFILL = synth.C4_PREFILL
@@ -325,14 +334,25 @@ class OracleQuery:
     of every key row can run on T host threads, each scoring a contiguous
     slice of the rows with the oracle's index_scores; BLAS gets T threads.
     The FP4 rows of each layer's attention set are stored by the oracle's
-    quantiser before the timed run (the cache write is not part of a step)."""
+    quantiser before the timed run (the cache write is not part of a step).
+    With ``local``, every layer reads its window from its own ring of bf16
+    rows (the oracle's kv_rows_local_window) and every reuse layer reads the
+    FP4 rows of the layer whose selection it reuses."""
 
-    def __init__(self, wl, query: int):
+    def __init__(self, wl, query: int, local: bool = False):
         import oracle as O
         self.O, self.wl = O, wl
         sq, qp = wl.query_positions()
         self.seq, self.pos = int(sq[query]), int(qp[query])
         n = self.pos + 1
+        self.rings = None
+        if local:   # ring of the query's sequence: position p in row p mod R
+            R, a = wl.window, max(0, n - wl.window)
+            self.rings = []
+            for l in range(len(wl.modes)):
+                ring = np.zeros((R, wl.attn_dim), np.float64)
+                ring[np.arange(a, n) % R] = synth.local_kv_values(wl, l, self.seq, a, n)
+                self.rings.append(ring)
         self.layers = []
         for l, mode in enumerate(wl.modes):
             d = {"q_attn": synth.attn_query(wl, l, query)}
@@ -350,10 +370,12 @@ class OracleQuery:
                 sel = O.top_k_positions(scores0[pool], pool, wl.topk)
             elif mode == synth.REINDEX:
                 _, sel = O.reindex(d["q"], d["w"], d["keys"], pool, wl.topk)
+            if mode != synth.REUSE or not local:
+                src = l   # the layer whose FP4 cache this layer reads
             S = O.attention_set(sel, self.pos, wl.window)
             codes = np.zeros((n, wl.attn_dim // 2), np.uint8)
             scales = np.zeros((n, wl.attn_dim // 32), np.uint8)
-            x = np.concatenate([synth.kv_values(wl, l, self.seq, int(r), int(r) + 1) for r in S])
+            x = np.concatenate([synth.kv_values(wl, src, self.seq, int(r), int(r) + 1) for r in S])
             codes[S], scales[S] = O.fp4_quantize(x)
             self.codes.append((codes, scales))
 
@@ -396,7 +418,11 @@ class OracleQuery:
                     _, sel = O.reindex(d["q"], d["w"], d["keys"], pool, wl.topk)
                 S = O.attention_set(sel, pos, wl.window)
                 codes, scales = self.codes[l]
-                O.sparse_attention(d["q_attn"], O.fp4_dequant(codes[S], scales[S], wl.attn_dim))
+                if self.rings is None:
+                    kv = O.fp4_dequant(codes[S], scales[S], wl.attn_dim)
+                else:
+                    kv = O.kv_rows_local_window(S, pos, wl.window, codes, scales, wl.attn_dim, self.rings[l])
+                O.sparse_attention(d["q_attn"], kv)
                 t_total += time.perf_counter() - t0
         return t_total
 
@@ -412,6 +438,9 @@ def oracle_sample(key: str):
     if key == "verify":
         q = len(qp) - 1
         return OracleQuery(wl, q), len(qp), "the block's last query (whole 1M prefix) through all 8 layers, x5 per block"
+    if key in LOCAL_WINDOW_WORKLOADS:
+        return (OracleQuery(wl, 0, local=True), 1,
+                f"one whole {len(wl.modes)}-layer decode step of the same workload (window rows from the local rings)")
     return OracleQuery(wl, 0), 1, f"one whole {len(wl.modes)}-layer decode step of the same workload"
 
 
@@ -477,6 +506,9 @@ def config_dict(key: str, wl, n_rep: int | None = None, rep_bytes: int | None = 
     if key == "verify":
         d["verify_block"] = f"{len(qp)} causal queries at positions {int(qp[0])}..{int(qp[-1])}, one sequence, " \
                             "index scan shared (group_queries)"
+    if key in LOCAL_WINDOW_WORKLOADS:
+        d["local_window"] = (f"every layer's last {wl.window} positions from its own bf16 ring of {wl.window} rows; "
+                             "reuse layers read the FP4 cache of the layer they reuse")
     if n_rep is not None:
         d["l2"] = (f"inputs rotate over {n_rep} device replicas ({rep_bytes * n_rep / 1e6:.0f} MB of caches, "
                    f"> L2)")
@@ -493,7 +525,7 @@ def run_decode(args, rank, world, local):
     torch.cuda.set_device(dev)
     t_setup = time.time()
     status = B.new_status(dev)
-    base = W.build_decode(wl, dev, status)
+    base = W.build_decode(wl, dev, status, local_window=key in LOCAL_WINDOW_WORKLOADS)
     rep_bytes = W.state_bytes(base)
     n_rep = args.replicas or max(4, min(MAX_REPLICAS, math.ceil(2 * l2_bytes(dev) / max(rep_bytes, 1))))
     replicas = [base] + [W.clone_decode(base, dev) for _ in range(n_rep - 1)]

@@ -106,10 +106,27 @@ def _key_rows(wl, layer, lens, pt, dev):
     return keys, 0
 
 
-def build_decode(wl: synth.Workload, dev, status) -> DecodeState:
+def local_ring_rows(wl: synth.Workload, layer: int, lens, R: int) -> np.ndarray:
+    """float32 [len(lens) * R][attn_dim] local window cache of one layer: a
+    ring of R rows per sequence, position p of sequence s in row s R + p mod R,
+    holding the last R positions (synth.local_kv_values)."""
+    rows = np.zeros((len(lens) * R, wl.attn_dim), np.float32)
+    for s, n in enumerate(lens):
+        n = int(n)
+        a = max(0, n - R)
+        rows[s * R + np.arange(a, n) % R] = synth.local_kv_values(wl, layer, s, a, n)
+    return rows
+
+
+def build_decode(wl: synth.Workload, dev, status, local_window: bool = False) -> DecodeState:
     """Builds one replica of a decode workload: one query per sequence at its
     last position, or a block of causal queries of sequence 0 when the
-    workload has a query block (a verify block)."""
+    workload has a query block (a verify block).
+
+    With ``local_window`` every layer reads its window from its own bf16
+    ring of ``wl.window`` rows per sequence, and every REUSE layer reads the
+    global FP4 cache of the layer whose selection it reuses (the same codes
+    and scales views)."""
     lens = wl.lengths()
     sq, qp = wl.query_positions()
     nq = len(qp)
@@ -131,13 +148,23 @@ def build_decode(wl: synth.Workload, dev, status) -> DecodeState:
     vin, vout = pin.views(inbuf), pout.views(outbuf)
 
     layers = []
+    src = 0   # the most recent FULL/REINDEX layer
     for l, mode in enumerate(wl.modes):
         s = slots[l]
         qa = vin[s["qa"]]
         qa.copy_(torch.from_numpy(np.stack([synth.attn_query(wl, l, i) for i in range(nq)])).to(torch.bfloat16))
-        codes, scales, srows = _fp4_rows(wl, l, lens, pt, dev, status)
-        ly = B.Layer(q_attn=qa, codes=B.Rows(codes, pt_dev, pr, srows), scales=B.Rows(scales, pt_dev, pr, srows),
-                     out=vout[s["out"]], lse=None)
+        if mode != synth.REUSE:
+            src = l
+        if local_window and mode == synth.REUSE:
+            ly = B.Layer(q_attn=qa, codes=layers[src].codes, scales=layers[src].scales, out=vout[s["out"]],
+                         lse=None)
+        else:
+            codes, scales, srows = _fp4_rows(wl, l, lens, pt, dev, status)
+            ly = B.Layer(q_attn=qa, codes=B.Rows(codes, pt_dev, pr, srows),
+                         scales=B.Rows(scales, pt_dev, pr, srows), out=vout[s["out"]], lse=None)
+        if local_window:
+            ring = torch.from_numpy(local_ring_rows(wl, l, lens, wl.window)).to(dev).to(torch.bfloat16)
+            ly.local_kv = B.Rows(ring, seq_rows=wl.window)
         if mode != synth.REUSE:
             keys, ksr = _key_rows(wl, l, lens, pt, dev)
             ly.keys = B.Rows(keys, pt_dev, pr, ksr)
@@ -161,15 +188,22 @@ def build_decode(wl: synth.Workload, dev, status) -> DecodeState:
 
 
 def clone_decode(st: DecodeState, dev) -> DecodeState:
-    """A second replica of the same state: every cache and buffer copied."""
+    """A second replica of the same state: every cache and buffer copied
+    (a cache that several layers share stays shared in the copy)."""
     inbuf, outbuf = st.inbuf.clone(), torch.zeros_like(st.outbuf)
     vin, vout = st.extra["pin"].views(inbuf), st.extra["pout"].views(outbuf)
+    copies = {}
+
+    def copy(r: "B.Rows") -> "B.Rows":
+        if id(r) not in copies:
+            copies[id(r)] = B.Rows(r.data.clone(), r.page_table, r.page_rows, r.seq_rows)
+        return copies[id(r)]
     layers = []
     for ly, s in zip(st.layers, st.extra["slots"]):
-        c = B.Layer(q_attn=vin[s["qa"]], out=vout[s["out"]], lse=None,
-                    codes=B.Rows(ly.codes.data.clone(), ly.codes.page_table, ly.codes.page_rows, ly.codes.seq_rows),
-                    scales=B.Rows(ly.scales.data.clone(), ly.scales.page_table, ly.scales.page_rows,
-                                  ly.scales.seq_rows))
+        c = B.Layer(q_attn=vin[s["qa"]], out=vout[s["out"]], lse=None, codes=copy(ly.codes),
+                    scales=copy(ly.scales))
+        if ly.local_kv is not None:
+            c.local_kv = copy(ly.local_kv)
         if ly.keys is not None:
             c.keys = B.Rows(ly.keys.data.clone(), ly.keys.page_table, ly.keys.page_rows, ly.keys.seq_rows)
             c.q, c.w = vin[s["q"]], vin[s["w"]]
@@ -189,12 +223,13 @@ def decode_plan(st: DecodeState, group_queries: bool = False) -> "B.LayerPlan":
 
 
 def state_bytes(st: DecodeState) -> int:
-    """Device bytes of the caches of one replica."""
-    n = 0
+    """Device bytes of the caches of one replica (a shared cache once)."""
+    seen, n = set(), 0
     for ly in st.layers:
-        n += ly.codes.data.numel() + ly.scales.data.numel()
-        if ly.keys is not None:
-            n += ly.keys.data.numel()
+        for r in (ly.codes, ly.scales, ly.keys, ly.local_kv):
+            if r is not None and id(r.data) not in seen:
+                seen.add(id(r.data))
+                n += r.data.numel() * r.data.element_size()
     return n
 
 
@@ -206,7 +241,8 @@ def algorithmic_bytes(st: DecodeState) -> tuple[int, dict]:
         share one scan);
       - per query and reindex layer, the key rows of the pool it gathers;
       - per query and layer, the FP4 rows of its attention set (selection and
-        window, each position once);
+        window, each position once), or with a local window cache the FP4
+        rows below the window and the window's bf16 rows;
       - queries, head weights and outputs.
     Scores, histograms and index lists are intermediates and are not counted."""
     wl = st.wl
@@ -232,10 +268,10 @@ def algorithmic_bytes(st: DecodeState) -> tuple[int, dict]:
             parts["q_w_out"] += len(qp) * (wl.idx_heads * wl.idx_dim + wl.idx_heads)
         if mode == synth.REINDEX:
             parts["reindex_gather"] += int(pool_cnt.sum()) * row_idx
+        row_win = 2 * wl.attn_dim if ly.local_kv is not None else row_fp4
         for i, p in enumerate(qp):
             wstart = max(0, int(p) - wl.window + 1)
-            n_s = int((sel_h[i] < wstart).sum()) + (int(p) - wstart + 1)
-            parts["attn_rows"] += n_s * row_fp4
+            parts["attn_rows"] += int((sel_h[i] < wstart).sum()) * row_fp4 + (int(p) - wstart + 1) * row_win
         parts["q_w_out"] += 2 * len(qp) * wl.attn_heads * wl.attn_dim * 2
     return sum(parts.values()), parts
 

@@ -27,6 +27,8 @@ def _bench():
 
 
 class _Layer:
+    local_kv = None
+
     def __init__(self, sels, pool_cnt=None):
         K = max(len(s) for s in sels)
         self.sel_idx = torch.tensor([list(s) + [-1] * (K - len(s)) for s in sels], dtype=torch.int32)
@@ -65,6 +67,37 @@ def test_window_overlap_is_counted_once():
     row_fp4 = wl.attn_dim // 2 + wl.attn_dim // 32
     below = 512 - wl.window                            # selected rows before the window start
     assert parts["attn_rows"] == 8 * (below + wl.window) * row_fp4
+
+
+def test_local_window_rows_are_counted_as_bf16():
+    """With a local window cache the window's rows are bf16 (2 bytes per
+    value) and only the selected rows below the window are FP4."""
+    bench = _bench()
+    wl = bench.WL_WINDOW
+    pos = int(wl.lengths()[0]) - 1
+    sel = list(range(0, 384 * 1000, 1000)) + list(range(pos - 127, pos + 1))   # 384 below, 128 in the window
+    st = _state(wl, [sel])
+    for ly in st.layers:
+        ly.local_kv = object()
+    _, parts = W.algorithmic_bytes(st)
+    row_fp4 = wl.attn_dim // 2 + wl.attn_dim // 32
+    assert parts["attn_rows"] == 8 * (384 * row_fp4 + wl.window * 2 * wl.attn_dim)
+    assert "window" in bench.LOCAL_WINDOW_WORKLOADS and bench.DECODE_WORKLOADS["window"][0] is wl
+
+
+def test_local_ring_places_the_last_positions():
+    """Ring row s R + p mod R holds position p of sequence s for the last R
+    positions (the other rows stay zero)."""
+    wl = synth.scaled(synth.C0_TINY, seq_lens=(300, 90))
+    R = 128
+    rows = W.local_ring_rows(wl, 0, wl.lengths(), R)
+    assert rows.shape == (2 * R, wl.attn_dim)
+    for s, n in enumerate(wl.lengths()):
+        a = max(0, int(n) - R)
+        x = synth.local_kv_values(wl, 0, s, a, int(n))
+        for p in range(a, int(n)):
+            assert np.array_equal(rows[s * R + p % R], x[p - a])
+    assert not rows[R + 90:2 * R].any()
 
 
 def test_verify_block_reads_the_keys_once_per_sequence():
